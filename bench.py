@@ -1,0 +1,405 @@
+"""Benchmark of the Star Attention hot path on B200 (one attention layer).
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+RoPE + Phase-1 anchor-block encoding of the context, the Phase-2 query chunk
+(partials + LSE merge), then every single-token decode step (partials + LSE
+merge). Inputs are resident in HBM when the timed region starts.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl star|reference]
+
+One JSON line on stdout (rank 0). With N > 1 (torchrun, one rank per GPU)
+each rank runs its own independent sequences (weak scaling, no data-path
+collective); the time is the max over ranks.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "Phase1 context tok/s + % bf16 TC peak; Phase2 decode tok/s + HBM GB/s (1 GPU)"
+DEFAULT_CONFIG = "llama8b-16k"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi during timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- oracle CPU baseline
+def oracle_sample(w, budget_s=15.0, seed=0):
+    """Times the fp64 oracle, as it stands, on a bounded random sample of the
+    workload: Phase-1 rows, and the Phase-2 rows of one decode step.
+    Returns an estimated step time (s) scaled to the whole step, and a label."""
+    import numpy as np
+    import torch
+
+    from block_sparse_long_rope_b200 import inputs
+    from oracle import oracle as orc
+
+    rng = np.random.default_rng(seed)
+    # Phase 1: random (head, row) pairs of sequence 0, uniform over rows
+    q, k, v = inputs.make_context(1, w.L, w.Hq, w.Hkv, w.D, w.index)
+    q2, k2, v2 = inputs.make_new_tokens(1, w.Tq + w.Tdec, w.Hq, w.Hkv, w.D, w.index)
+    rows_done, t_p1 = 0, 0.0
+    batch = 32
+    while t_p1 < budget_s * 0.7:
+        rows = rng.integers(0, w.L, size=batch)
+        heads = rng.integers(0, w.Hq, size=batch)
+        t0 = time.perf_counter()
+        orc.phase1_rows(q, k, v, w.block_len, w.anchor_len, w.theta, np.zeros(batch), heads, rows)
+        t_p1 += time.perf_counter() - t0
+        rows_done += batch
+    per_row_p1 = t_p1 / rows_done
+    # Phase 2: all heads of one decode token (every split) at the end of the tail
+    tail = w.Tq + w.Tdec - 1
+    t0 = time.perf_counter()
+    orc.phase2_rows(q2[:, tail:tail + 1], k, v, k2, v2, w.block_len, tail, w.theta,
+                    np.zeros(w.Hq), np.arange(w.Hq), np.zeros(w.Hq))
+    t_dec = time.perf_counter() - t0  # one decode token, all heads
+    est_step = (per_row_p1 * w.L * w.Hq + t_dec * (w.Tq + w.Tdec)) * w.B
+    sample = (f"{rows_done} random Phase-1 (row, head) queries of sequence 0 and one decode token "
+              f"(all {w.Hq} heads, all splits); step time extrapolated to B*L*Hq Phase-1 rows and "
+              f"Tq+Tdec Phase-2 tokens")
+    del q, k, v, q2, k2, v2, torch
+    return est_step, sample, t_p1 + t_dec
+
+
+def omp_threads():
+    v = os.environ.get("OMP_NUM_THREADS")
+    return int(v) if v else (os.cpu_count() or 1)
+
+
+# --------------------------------------------------------------------------- star arm
+def run_star(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from block_sparse_long_rope_b200 import inputs, star
+    from block_sparse_long_rope_b200.pipeline import StarLayer, phase2_calls
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks, peak_src = load_peaks()
+
+    # inputs: every rank holds its own independent sequences (seeded per rank)
+    cfg_index = w.index + 100 * rank
+    with torch.no_grad():
+        ctx = inputs.make_context(w.B, w.L, w.Hq, w.Hkv, w.D, cfg_index, device=dev)
+        new = inputs.make_new_tokens(w.B, w.Tq + w.Tdec, w.Hq, w.Hkv, w.D, cfg_index, device=dev)
+    calls = phase2_calls(w, *new)
+    layer = StarLayer(w, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        layer.encode(*ctx)
+        if ev is not None:
+            ev[1].record(stream)
+        q2, k2, v2, tail = calls[0]
+        layer.attend(q2, k2, v2, tail)
+        if ev is not None:
+            ev[2].record(stream)
+        for (q2, k2, v2, tail) in calls[1:]:
+            layer.attend(q2, k2, v2, tail)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    star.star_device_status(layer.buf.ws1)
+    star.star_device_status(layer.buf.ws2)
+    torch.cuda.synchronize()
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    elapsed_ms = start.elapsed_time(end)
+    p1_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    chunk_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    dec_ms = sum(e[2].elapsed_time(e[3]) for e in evs)
+    star.star_device_status(layer.buf.ws1)
+    star.star_device_status(layer.buf.ws2)
+
+    if world > 1:
+        t = torch.tensor([elapsed_ms, p1_ms, chunk_ms, dec_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed_ms, p1_ms, chunk_ms, dec_ms = t.tolist()
+
+    # ---- end to end through the public API with host buffers ----------------
+    host_ctx = [t.cpu().pin_memory() for t in ctx]
+    host_calls = [tuple(x.cpu().pin_memory() for x in c[:3]) + (c[3],) for c in calls]
+    dev_ctx = [torch.empty_like(t) for t in ctx]
+    dev_calls = [tuple(torch.empty_like(x) for x in c[:3]) + (c[3],) for c in calls]
+    host_o = torch.empty(layer.buf.o.shape, dtype=torch.bfloat16).pin_memory()
+    host_dec = torch.empty((w.B, 1, w.Hq, w.D), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_ctx) + \
+        sum(x.numel() * x.element_size() for c in host_calls for x in c[:3])
+    d2h = host_o.numel() * 2 + host_dec.numel() * 2
+
+    def e2e_step():
+        for d, h in zip(dev_ctx, host_ctx):
+            d.copy_(h, non_blocking=True)
+        for dc, hc in zip(dev_calls, host_calls):
+            for d, h in zip(dc[:3], hc[:3]):
+                d.copy_(h, non_blocking=True)
+        layer.encode(*dev_ctx)
+        out = None
+        for (q2, k2, v2, tail) in dev_calls:
+            out = layer.attend(q2, k2, v2, tail)
+        host_o.copy_(layer.buf.o, non_blocking=True)
+        host_dec.copy_(out[0], non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    s2 = torch.cuda.Event(enable_timing=True)
+    e2 = torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = s2.elapsed_time(e2)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+
+    if rank != 0:
+        return None
+
+    K = args.steps
+    ms_step = elapsed_ms / K
+    ctx_tokens = w.B * w.L * world
+    value = ctx_tokens / (ms_step / 1e3)
+    p1_s = p1_ms / K / 1e3
+    p1_flops = w.phase1_flops()
+    p1_tflops = p1_flops / p1_s / 1e12
+    bf16_peak = float(peaks["bf16_tflops"])
+    hbm_peak = float(peaks["hbm_gbs"])
+    dec_s = dec_ms / K / 1e3
+    # bytes of K+V cache every decode step reads (tail grows by one per step)
+    dec_bytes = sum(w.decode_kv_bytes(w.Tq + s) for s in range(w.Tdec))
+    dec_gbs = dec_bytes / dec_s / 1e9 if dec_s > 0 else None
+    dec_tok_s = w.B * w.Tdec / dec_s if dec_s > 0 else None
+    chunk_s = chunk_ms / K / 1e3
+    launches = 2 + 3 + 4 * w.Tdec  # rope+attn; rope+attn+merge; (rope+decode+reduce+merge) x Tdec
+
+    line = {
+        "metric": METRIC,
+        "value": round(value, 1),
+        "unit": "tok/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic N(0,1) bf16 Q/K/V (seeded); the pages' RULER/BABILong/InfiniteBench "
+                "runs need datasets and trained weights not available here",
+        "config": {
+            "workload": w.name, "B": w.B, "L": w.L, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+            "block_len": w.block_len, "anchor_len": w.anchor_len, "theta": w.theta,
+            "Tq": w.Tq, "Tdec": w.Tdec, "global_batch": w.B * world, "seq_len": w.L,
+            "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "step inputs (Q+K+V context, 192 MiB at 16K) exceed the 126 MB L2; no flush",
+        },
+        "phases": {
+            "phase1": {"ms": round(p1_s * 1e3, 4), "ctx_tok_s": round(w.B * w.L / p1_s, 1),
+                       "unmasked_tflops": round(p1_tflops, 2),
+                       "frac_bf16_peak": round(p1_tflops / bf16_peak, 4),
+                       "note": "star_phase1_encode call: RoPE kernel + attention kernel"},
+            "phase2_query_chunk": {"ms": round(chunk_s * 1e3, 4), "tokens": w.Tq,
+                                   "tflops": round(4.0 * w.D * w.Hq * w.B * w.Tq * w.L / chunk_s / 1e12, 2)},
+            "phase2_decode": {"ms": round(dec_s * 1e3, 4), "tok_s": round(dec_tok_s, 1),
+                              "kv_gbs": round(dec_gbs, 1),
+                              "frac_hbm": round(dec_gbs / hbm_peak, 4),
+                              "note": "per step: RoPE/append + split-KV decode + split reduce + "
+                                      "merge; K/V just written by Phase 1, so a 16K cache "
+                                      "(64 MiB) is partly L2-resident"},
+        },
+        "roofline": {"bound": "tensor", "kernel": "phase1 (star_phase1_encode)",
+                     "achieved": round(p1_tflops, 2), "peak": bf16_peak,
+                     "unit": "TFLOP/s", "frac": round(p1_tflops / bf16_peak, 4),
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "algorithmic": "4*D*Hq*B*[n*b(b+1)/2 + (n-1)*a*b] unmasked FLOPs per launch "
+                                    f"= {p1_flops:.4g}",
+                     "traffic": None},
+        "e2e": {"value": round(ctx_tokens / (e2e_ms / K / 1e3), 1), "unit": "tok/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": launches * K,
+        "clocks": clocks,
+    }
+    if args.cpu_baseline:
+        est_step, sample, spent = oracle_sample(w, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(w.B * w.L / est_step, 3), "unit": "tok/s",
+                                "cores": omp_threads(), "kind": "oracle", "sample": sample,
+                                "seconds_spent": round(spent, 2), "extrapolated": True}
+    return line
+
+
+def run_reference(args, w, rank):
+    """Reference arm: the fp64 oracle as it stands, on the host cores, each step
+    a bounded sample of the workload scaled to the step."""
+    if rank != 0:
+        return None
+    for _ in range(args.warmup):
+        oracle_sample(w, budget_s=0.5)
+    t0 = time.perf_counter()
+    est = []
+    sample = ""
+    for _ in range(args.steps):
+        e, sample, _ = oracle_sample(w, budget_s=args.ref_budget)
+        est.append(e)
+    wall = time.perf_counter() - t0
+    est_step = sum(est) / len(est)
+    value = w.B * w.L / est_step
+    return {
+        "metric": METRIC, "value": round(value, 3), "unit": "tok/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(est_step * 1e3, 1),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic N(0,1) bf16 Q/K/V (seeded)", "impl": "reference",
+        "config": {"workload": w.name, "B": w.B, "L": w.L, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+                   "block_len": w.block_len, "anchor_len": w.anchor_len},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tok/s", "cores": omp_threads(),
+                         "kind": "oracle", "sample": sample, "extrapolated": True},
+        "e2e": {"value": round(value, 3), "unit": "tok/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": round(wall, 2),
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default=DEFAULT_CONFIG)
+    ap.add_argument("--impl", default="star", choices=["star", "reference"])
+    ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=8.0)
+    args = ap.parse_args()
+
+    from block_sparse_long_rope_b200.configs import BY_NAME
+    w = BY_NAME[args.config]
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        backend = "nccl" if args.impl == "star" else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, w, rank)
+        else:
+            line = run_star(args, w, rank, world, local_rank)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

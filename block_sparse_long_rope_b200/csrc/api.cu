@@ -1,0 +1,493 @@
+// C ABI of the Star Attention hot path (declared in include/star.h):
+// argument validation, workspace layout, TMA descriptor encoding and kernel
+// launches on the caller's stream. No allocation, no synchronisation (except
+// star_device_status).
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+
+#include "../../include/star.h"
+#include "star_common.cuh"
+#include "star_kernels.cuh"
+
+namespace {
+
+using star::ceil_div;
+using star::imin;
+
+thread_local std::string g_err;
+
+star_status fail(star_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return s;
+}
+
+star_status ok() {
+  g_err.clear();
+  return STAR_OK;
+}
+
+star_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(STAR_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- device properties (cached per device) ----------------------------------
+struct DevInfo {
+  bool probed = false, supported = false;
+  int sms = 0;
+  char name[128] = {0};
+};
+DevInfo g_dev[64];
+std::mutex g_dev_mu;
+
+star_status check_device(int* num_sms) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(STAR_ERR_UNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DevInfo& d = g_dev[dev];
+  if (!d.probed) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+    d.supported = (major == 10 && minor == 0);
+    snprintf(d.name, sizeof d.name, "sm_%d%d", major, minor);
+    d.probed = true;
+  }
+  if (!d.supported)
+    return fail(STAR_ERR_UNSUPPORTED, "device %d is %s; this library is built for sm_100a (B200)",
+                dev, d.name);
+  if (num_sms) *num_sms = d.sms;
+  return STAR_OK;
+}
+
+// ---- TMA descriptors ------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// rank-4 map over a token-major [B, rows, H, D] bf16 buffer; box {64, 1, 128, 1}
+star_status map_token_major(CUtensorMap* m, const void* base, int B, int rows, int H, int D) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(STAR_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)B};
+  cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)rows * H * D * 2};
+  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t es[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(STAR_ERR_CUDA, "cuTensorMapEncodeTiled(Q) failed: %d", (int)r);
+  return STAR_OK;
+}
+
+// rank-3 map over a head-major cache [B*Hkv, Lcap, D], rows [0, valid) visible;
+// box {64, box_rows, 1}
+star_status map_cache(CUtensorMap* m, const void* base, int BH, int Lcap, int valid, int D,
+                      int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return fail(STAR_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)valid, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)Lcap * D * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                   box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(STAR_ERR_CUDA, "cuTensorMapEncodeTiled(cache) failed: %d", (int)r);
+  return STAR_OK;
+}
+
+// ---- shared argument checks ----------------------------------------------------
+star_status check_heads(int B, int Hq, int Hkv, int D) {
+  if (B < 1 || Hq < 1 || Hkv < 1) return fail(STAR_ERR_INVALID_ARG, "B, Hq, Hkv must be >= 1");
+  if (Hq % Hkv != 0) return fail(STAR_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
+  if (D != 64 && D != 128) return fail(STAR_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", D);
+  return STAR_OK;
+}
+
+star_status check_ptr(const void* p, const char* name) {
+  if (!p) return fail(STAR_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!aligned16(p)) return fail(STAR_ERR_INVALID_ARG, "%s is not 16-byte aligned", name);
+  return STAR_OK;
+}
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+// Decode path scratch: per (batch, KV head), chunk partials of kDecRows rows.
+int decode_chunks_per_head(int L, int b, int n, int tail_plus_T, int chunk, int* nc_full,
+                           int* nc_last, int* nc_tail) {
+  *nc_full = ceil_div(imin(b, L), chunk);
+  *nc_last = ceil_div(L - (n - 1) * b, chunk);
+  *nc_tail = ceil_div(tail_plus_T, chunk);
+  return (n - 1) * *nc_full + *nc_last + *nc_tail;
+}
+constexpr int kMinChunk = 256;
+constexpr int kMaxChunk = 4096;
+
+bool use_decode_path(int T, int Hq, int Hkv) {
+  const int g = Hq / Hkv;
+  return T * g <= star::kDecRows;
+}
+
+size_t decode_scratch_bytes(int B, int Hkv, int D, int Lcap, int block_len) {
+  // worst case over L + tail <= Lcap at the smallest chunk
+  const long long nsplit_max = ceil_div(Lcap, block_len) + 1;
+  const long long cph = ceil_div(Lcap, kMinChunk) + nsplit_max;
+  const long long rows = (long long)B * Hkv * cph * star::kDecRows;
+  return align_up((size_t)rows * D * sizeof(float)) + align_up((size_t)rows * sizeof(float));
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* star_last_error(void) { return g_err.c_str(); }
+
+const char* star_version(void) { return "star-b200 0.1 (sm_100a)"; }
+
+star_status star_rope(const void* x, const int64_t x_stride[3], void* y, const int64_t y_stride[3],
+                      const int32_t* pos, int64_t pos0, int B, int S, int H, int D, double theta,
+                      void* cuda_stream) {
+  if (!x_stride || !y_stride) return fail(STAR_ERR_INVALID_ARG, "stride arrays are NULL");
+  if (B < 0 || S < 0 || H < 1) return fail(STAR_ERR_INVALID_ARG, "bad shape B=%d S=%d H=%d", B, S, H);
+  if (D != 64 && D != 128) return fail(STAR_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", D);
+  if (!(theta > 0.0)) return fail(STAR_ERR_INVALID_ARG, "theta must be > 0");
+  star_status s;
+  if ((s = check_ptr(x, "x")) != STAR_OK || (s = check_ptr(y, "y")) != STAR_OK) return s;
+  for (int i = 0; i < 3; ++i)
+    if (x_stride[i] % 8 != 0 || y_stride[i] % 8 != 0)
+      return fail(STAR_ERR_INVALID_ARG, "strides must be multiples of 8 elements");
+  if (pos && (reinterpret_cast<uintptr_t>(pos) & 3u))
+    return fail(STAR_ERR_INVALID_ARG, "pos is not 4-byte aligned");
+  if ((s = check_device(nullptr)) != STAR_OK) return s;
+  if (B == 0 || S == 0) return ok();
+  star::RopeParams p{};
+  p.job[0] = star::RopeJob{static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y),
+                           {x_stride[0], x_stride[1], x_stride[2]},
+                           {y_stride[0], y_stride[1], y_stride[2]}, H, 1};
+  p.B = B;
+  p.S = S;
+  p.D = D;
+  p.pos = pos;
+  p.pos0 = pos0;
+  star::rope_set_freq(p, D, theta);
+  cudaError_t e = star::launch_rope(p, 1, static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return cuda_fail(e, "rope launch");
+  return ok();
+}
+
+size_t star_phase1_workspace_bytes(int B, int L, int Hq, int D) {
+  if (B < 1 || L < 1 || Hq < 1 || D < 1) return star::kStatusBytes;
+  return star::kStatusBytes + align_up((size_t)B * L * Hq * D * 2);
+}
+
+star_status star_phase1_encode(const void* q, const void* k, const void* v, void* o, void* k_cache,
+                               void* v_cache, int Lcap, float* lse, int B, int L, int Hq, int Hkv,
+                               int D, int block_len, int anchor_len, double theta, void* workspace,
+                               size_t workspace_bytes, void* cuda_stream) {
+  star_status s;
+  if ((s = check_heads(B, Hq, Hkv, D)) != STAR_OK) return s;
+  if (L < 1) return fail(STAR_ERR_INVALID_ARG, "L must be >= 1");
+  if (block_len < 1) return fail(STAR_ERR_INVALID_ARG, "block_len must be >= 1");
+  if (anchor_len < 0 || anchor_len > block_len)
+    return fail(STAR_ERR_INVALID_ARG, "anchor_len (%d) must lie in [0, block_len=%d]", anchor_len,
+                block_len);
+  if (Lcap < L) return fail(STAR_ERR_INVALID_ARG, "Lcap (%d) < L (%d)", Lcap, L);
+  if (!(theta > 0.0)) return fail(STAR_ERR_INVALID_ARG, "theta must be > 0");
+  if ((s = check_ptr(q, "q")) || (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) ||
+      (s = check_ptr(o, "o")) || (s = check_ptr(k_cache, "k_cache")) ||
+      (s = check_ptr(v_cache, "v_cache")) || (s = check_ptr(workspace, "workspace")))
+    return s;
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(STAR_ERR_INVALID_ARG, "lse is not 4-byte aligned");
+  const size_t need = star_phase1_workspace_bytes(B, L, Hq, D);
+  if (workspace_bytes < need)
+    return fail(STAR_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+  if ((long long)B * Hkv > (1ll << 31) - 1) return fail(STAR_ERR_INVALID_ARG, "B*Hkv too large");
+  if ((s = check_device(nullptr)) != STAR_OK) return s;
+
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  __nv_bfloat16* qrot = reinterpret_cast<__nv_bfloat16*>(ws + star::kStatusBytes);
+  cudaError_t e = cudaMemsetAsync(ws, 0, star::kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "status reset");
+
+  // RoPE: Q -> workspace (token-major), K -> k_cache (head-major, rotated),
+  // V -> v_cache (head-major copy). Token t sits at position t.
+  star::RopeParams rp{};
+  const long long qs[3] = {(long long)L * Hq * D, (long long)Hq * D, D};
+  const long long ks[3] = {(long long)L * Hkv * D, (long long)Hkv * D, D};
+  const long long cs[3] = {(long long)Hkv * Lcap * D, D, (long long)Lcap * D};
+  rp.job[0] = star::RopeJob{static_cast<const __nv_bfloat16*>(q), qrot, {qs[0], qs[1], qs[2]},
+                            {qs[0], qs[1], qs[2]}, Hq, 1};
+  rp.job[1] = star::RopeJob{static_cast<const __nv_bfloat16*>(k),
+                            static_cast<__nv_bfloat16*>(k_cache), {ks[0], ks[1], ks[2]},
+                            {cs[0], cs[1], cs[2]}, Hkv, 1};
+  rp.job[2] = star::RopeJob{static_cast<const __nv_bfloat16*>(v),
+                            static_cast<__nv_bfloat16*>(v_cache), {ks[0], ks[1], ks[2]},
+                            {cs[0], cs[1], cs[2]}, Hkv, 0};
+  rp.B = B;
+  rp.S = L;
+  rp.D = D;
+  rp.pos = nullptr;
+  rp.pos0 = 0;
+  star::rope_set_freq(rp, D, theta);
+  e = star::launch_rope(rp, 3, st);
+  if (e != cudaSuccess) return cuda_fail(e, "rope launch");
+
+  star::AttnParams ap;
+  memset(&ap, 0, sizeof ap);
+  if ((s = map_token_major(&ap.tmQ, qrot, B, L, Hq, D)) != STAR_OK) return s;
+  if ((s = map_cache(&ap.tmK, k_cache, B * Hkv, Lcap, L, D, 128)) != STAR_OK) return s;
+  if ((s = map_cache(&ap.tmV, v_cache, B * Hkv, Lcap, L, D, 128)) != STAR_OK) return s;
+  const int g = Hq / Hkv;
+  ap.geom.B = B;
+  ap.geom.Hq = Hq;
+  ap.geom.Hkv = Hkv;
+  ap.geom.hpc = (g % 2 == 0) ? 2 : 1;
+  ap.geom.L = L;
+  ap.geom.b = block_len;
+  ap.geom.a = anchor_len;
+  ap.geom.n = ceil_div(L, block_len);
+  ap.geom.T = 0;
+  ap.geom.tail_len = 0;
+  ap.mode = 0;
+  const long long items = (long long)ap.geom.phase1_items();
+  if (items > (1ll << 31) - 1) return fail(STAR_ERR_INVALID_ARG, "problem too large");
+  ap.num_items = (int)items;
+  ap.qrows = L;
+  ap.nsplit = 0;
+  ap.o = static_cast<__nv_bfloat16*>(o);
+  ap.lse = lse;
+  ap.status = reinterpret_cast<int*>(ws);
+  ap.scale_ln = (float)(1.0 / sqrt((double)D));
+  ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+  e = star::launch_attn(ap, D, st);
+  if (e != cudaSuccess) return cuda_fail(e, "phase-1 attention launch");
+  return ok();
+}
+
+size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lcap, int block_len) {
+  if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || D < 1 || Lcap < 1 || block_len < 1 || Hq % Hkv)
+    return star::kStatusBytes;
+  size_t bytes = star::kStatusBytes + align_up((size_t)B * T * Hq * D * 2);
+  if (use_decode_path(T, Hq, Hkv)) bytes += decode_scratch_bytes(B, Hkv, D, Lcap, block_len);
+  return bytes;
+}
+
+star_status star_phase2_partial(const void* q, const void* k, const void* v, int T, void* k_cache,
+                                void* v_cache, int Lcap, int L, int block_len, int tail_len,
+                                float* part_o, float* part_lse, int* nsplit_out, int B, int Hq,
+                                int Hkv, int D, double theta, void* workspace,
+                                size_t workspace_bytes, void* cuda_stream) {
+  star_status s;
+  if ((s = check_heads(B, Hq, Hkv, D)) != STAR_OK) return s;
+  if (T < 1) return fail(STAR_ERR_INVALID_ARG, "T must be >= 1");
+  if (L < 1) return fail(STAR_ERR_INVALID_ARG, "L must be >= 1");
+  if (block_len < 1) return fail(STAR_ERR_INVALID_ARG, "block_len must be >= 1");
+  if (tail_len < 0) return fail(STAR_ERR_INVALID_ARG, "tail_len must be >= 0");
+  if ((long long)L + tail_len + T > Lcap)
+    return fail(STAR_ERR_INVALID_ARG, "Lcap (%d) < L + tail_len + T (%lld)", Lcap,
+                (long long)L + tail_len + T);
+  if (!(theta > 0.0)) return fail(STAR_ERR_INVALID_ARG, "theta must be > 0");
+  if ((s = check_ptr(q, "q")) || (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) ||
+      (s = check_ptr(k_cache, "k_cache")) || (s = check_ptr(v_cache, "v_cache")) ||
+      (s = check_ptr(part_o, "part_o")) || (s = check_ptr(workspace, "workspace")))
+    return s;
+  if (!part_lse || (reinterpret_cast<uintptr_t>(part_lse) & 3u))
+    return fail(STAR_ERR_INVALID_ARG, "part_lse is NULL or not 4-byte aligned");
+  const size_t need = star_phase2_workspace_bytes(B, T, Hq, Hkv, D, Lcap, block_len);
+  if (workspace_bytes < need)
+    return fail(STAR_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
+  int sms = 148;
+  if ((s = check_device(&sms)) != STAR_OK) return s;
+
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  __nv_bfloat16* qrot = reinterpret_cast<__nv_bfloat16*>(ws + star::kStatusBytes);
+  const size_t qrot_bytes = align_up((size_t)B * T * Hq * D * 2);
+  cudaError_t e = cudaMemsetAsync(ws, 0, star::kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "status reset");
+
+  // RoPE of the new tokens at positions L + tail_len + t; K/V appended to the
+  // cache rows of the same index.
+  const int row0 = L + tail_len;
+  star::RopeParams rp{};
+  const long long qs[3] = {(long long)T * Hq * D, (long long)Hq * D, D};
+  const long long ks[3] = {(long long)T * Hkv * D, (long long)Hkv * D, D};
+  const long long cs[3] = {(long long)Hkv * Lcap * D, D, (long long)Lcap * D};
+  rp.job[0] = star::RopeJob{static_cast<const __nv_bfloat16*>(q), qrot, {qs[0], qs[1], qs[2]},
+                            {qs[0], qs[1], qs[2]}, Hq, 1};
+  rp.job[1] = star::RopeJob{static_cast<const __nv_bfloat16*>(k),
+                            static_cast<__nv_bfloat16*>(k_cache) + (size_t)row0 * D,
+                            {ks[0], ks[1], ks[2]}, {cs[0], cs[1], cs[2]}, Hkv, 1};
+  rp.job[2] = star::RopeJob{static_cast<const __nv_bfloat16*>(v),
+                            static_cast<__nv_bfloat16*>(v_cache) + (size_t)row0 * D,
+                            {ks[0], ks[1], ks[2]}, {cs[0], cs[1], cs[2]}, Hkv, 0};
+  rp.B = B;
+  rp.S = T;
+  rp.D = D;
+  rp.pos = nullptr;
+  rp.pos0 = row0;
+  star::rope_set_freq(rp, D, theta);
+  e = star::launch_rope(rp, 3, st);
+  if (e != cudaSuccess) return cuda_fail(e, "rope launch");
+
+  const int n = ceil_div(L, block_len);
+  const int nsplit = n + 1;
+  const int valid = L + tail_len + T;
+  const int g = Hq / Hkv;
+  if (nsplit_out) *nsplit_out = nsplit;
+
+  if (use_decode_path(T, Hq, Hkv)) {
+    star::DecodeParams dp;
+    memset(&dp, 0, sizeof dp);
+    if ((s = map_cache(&dp.tmK, k_cache, B * Hkv, Lcap, valid, D, star::kDecTile)) != STAR_OK) return s;
+    if ((s = map_cache(&dp.tmV, v_cache, B * Hkv, Lcap, valid, D, star::kDecTile)) != STAR_OK) return s;
+    dp.q = qrot;
+    dp.B = B;
+    dp.T = T;
+    dp.Hq = Hq;
+    dp.Hkv = Hkv;
+    dp.g = g;
+    dp.R = T * g;
+    dp.L = L;
+    dp.b = block_len;
+    dp.n = n;
+    dp.tail_len = tail_len;
+    // smallest chunk that still gives every SM several CTAs
+    int chunk = kMinChunk;
+    int nf, nl, nt;
+    while (chunk < kMaxChunk &&
+           (long long)B * Hkv * decode_chunks_per_head(L, block_len, n, tail_len + T, chunk * 2, &nf, &nl, &nt) >=
+               8ll * sms)
+      chunk *= 2;
+    dp.chunk = chunk;
+    dp.chunks_per_head = decode_chunks_per_head(L, block_len, n, tail_len + T, chunk, &dp.nc_full,
+                                                &dp.nc_last, &dp.nc_tail);
+    const size_t rows = (size_t)B * Hkv * dp.chunks_per_head * star::kDecRows;
+    dp.ws_o = reinterpret_cast<float*>(ws + star::kStatusBytes + qrot_bytes);
+    dp.ws_lse = reinterpret_cast<float*>(ws + star::kStatusBytes + qrot_bytes +
+                                         align_up(rows * D * sizeof(float)));
+    dp.part_o = part_o;
+    dp.part_lse = part_lse;
+    dp.status = reinterpret_cast<int*>(ws);
+    dp.scale_ln = (float)(1.0 / sqrt((double)D));
+    dp.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+    e = star::launch_decode(dp, D, st);
+    if (e != cudaSuccess) return cuda_fail(e, "phase-2 decode launch");
+    return ok();
+  }
+
+  star::AttnParams ap;
+  memset(&ap, 0, sizeof ap);
+  if ((s = map_token_major(&ap.tmQ, qrot, B, T, Hq, D)) != STAR_OK) return s;
+  if ((s = map_cache(&ap.tmK, k_cache, B * Hkv, Lcap, valid, D, 128)) != STAR_OK) return s;
+  if ((s = map_cache(&ap.tmV, v_cache, B * Hkv, Lcap, valid, D, 128)) != STAR_OK) return s;
+  ap.geom.B = B;
+  ap.geom.Hq = Hq;
+  ap.geom.Hkv = Hkv;
+  ap.geom.hpc = (g % 2 == 0) ? 2 : 1;
+  ap.geom.L = L;
+  ap.geom.b = block_len;
+  ap.geom.a = 0;
+  ap.geom.n = n;
+  ap.geom.T = T;
+  ap.geom.tail_len = tail_len;
+  ap.mode = 1;
+  ap.num_items = ap.geom.phase2_items();
+  ap.qrows = T;
+  ap.nsplit = nsplit;
+  ap.part_o = part_o;
+  ap.part_lse = part_lse;
+  ap.status = reinterpret_cast<int*>(ws);
+  ap.scale_ln = (float)(1.0 / sqrt((double)D));
+  ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
+  e = star::launch_attn(ap, D, st);
+  if (e != cudaSuccess) return cuda_fail(e, "phase-2 chunk attention launch");
+  return ok();
+}
+
+star_status star_lse_merge(const float* part_o, const float* part_lse, int nsplit, void* o,
+                           float* lse, int B, int T, int Hq, int D, void* cuda_stream) {
+  if (nsplit < 1 || B < 1 || T < 1 || Hq < 1)
+    return fail(STAR_ERR_INVALID_ARG, "bad shape nsplit=%d B=%d T=%d Hq=%d", nsplit, B, T, Hq);
+  if (D != 64 && D != 128) return fail(STAR_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", D);
+  star_status s;
+  if ((s = check_ptr(part_o, "part_o")) || (s = check_ptr(o, "o"))) return s;
+  if (!part_lse || (reinterpret_cast<uintptr_t>(part_lse) & 3u))
+    return fail(STAR_ERR_INVALID_ARG, "part_lse is NULL or not 4-byte aligned");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(STAR_ERR_INVALID_ARG, "lse is not 4-byte aligned");
+  if ((s = check_device(nullptr)) != STAR_OK) return s;
+  cudaError_t e = star::launch_lse_merge(part_o, part_lse, nsplit, static_cast<__nv_bfloat16*>(o),
+                                         lse, B, T, Hq, D, static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
+  return ok();
+}
+
+star_status star_device_status(void* workspace, void* cuda_stream) {
+  if (!workspace) return fail(STAR_ERR_INVALID_ARG, "workspace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
+  int word = 0;
+  e = cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "status read");
+  e = cudaMemset(workspace, 0, sizeof word);
+  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  if (word & star::kDevTimeout)
+    return fail(STAR_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait gave up (status 0x%x)", word);
+  if (word & star::kDevBounds)
+    return fail(STAR_ERR_DEVICE_BOUNDS, "a kernel found an index outside its buffer (status 0x%x)", word);
+  return ok();
+}
+
+star_status star_debug_index(int L, int block_len, int anchor_len, int32_t* blk, int32_t* pos,
+                             int32_t* kv_ranges, void* cuda_stream) {
+  if (L < 1 || block_len < 1 || anchor_len < 0 || anchor_len > block_len)
+    return fail(STAR_ERR_INVALID_ARG, "bad L/block_len/anchor_len");
+  star_status s;
+  if ((s = check_ptr(blk, "blk")) || (s = check_ptr(pos, "pos")) || (s = check_ptr(kv_ranges, "kv_ranges")))
+    return s;
+  if ((s = check_device(nullptr)) != STAR_OK) return s;
+  cudaError_t e = star::launch_debug_index(L, block_len, anchor_len, blk, pos, kv_ranges,
+                                           static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return cuda_fail(e, "debug index launch");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,111 @@
+// Exact merge of per-split partials into global attention.
+//
+// Each split h carries a softmax-normalised output o_h and its log-sum-exp
+// lse_h. The pages' corrected online-softmax update weights a split by
+// exp(s_h - s_global) [pith 2WVXFXZ2, minor comment on Algorithm 2]; with
+// m = max_h lse_h this is
+//   w_h = exp(lse_h - m),  o = sum_h w_h o_h / sum_h w_h,  lse = m + log(sum_h w_h)
+// which reproduces softmax over the concatenated keys exactly [pith 2WVXFXZ2,
+// assumptions: online softmax aggregation yields the exact global softmax].
+//
+// One warp per (batch, head, token) row; lanes cover D with 16-byte loads.
+// HBM-bound and tiny: it reads nsplit * (D + 1) floats per row.
+#include <math.h>
+
+#include "star_common.cuh"
+#include "star_kernels.cuh"
+
+namespace star {
+
+template <int D>
+__global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict__ part_o,
+                                                        const float* __restrict__ part_lse,
+                                                        int nsplit, __nv_bfloat16* __restrict__ o,
+                                                        float* __restrict__ lse, int B, int T,
+                                                        int Hq) {
+  constexpr int kPer = D / 32;  // floats per lane (2 or 4)
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  const int rows = B * Hq * T;
+  if (warp >= rows) return;
+  const int t = warp % T;
+  const int h = (warp / T) % Hq;
+  const int b = warp / (T * Hq);
+  const size_t bh = static_cast<size_t>(b) * Hq + h;
+
+  float m = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) m = fmaxf(m, part_lse[(bh * nsplit + s) * T + t]);
+  float acc[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) acc[j] = 0.f;
+  float z = 0.f;
+  if (m != -INFINITY) {
+    for (int s = 0; s < nsplit; ++s) {
+      float l = part_lse[(bh * nsplit + s) * T + t];
+      if (l == -INFINITY) continue;
+      float w = expf(l - m);
+      z += w;
+      const float* src = part_o + ((bh * nsplit + s) * T + t) * D + lane * kPer;
+      if constexpr (kPer == 4) {
+        float4 v = *reinterpret_cast<const float4*>(src);
+        acc[0] += w * v.x;
+        acc[1] += w * v.y;
+        acc[2] += w * v.z;
+        acc[3] += w * v.w;
+      } else {
+        float2 v = *reinterpret_cast<const float2*>(src);
+        acc[0] += w * v.x;
+        acc[1] += w * v.y;
+      }
+    }
+  }
+  const float inv = (z > 0.f) ? 1.f / z : 0.f;
+  __nv_bfloat16* dst = o + ((static_cast<size_t>(b) * T + t) * Hq + h) * D + lane * kPer;
+  if constexpr (kPer == 4) {
+    uint2 pk;
+    pk.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    pk.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(dst) = pk;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  }
+  if (lse != nullptr && lane == 0) lse[bh * T + t] = (z > 0.f) ? m + logf(z) : -INFINITY;
+}
+
+cudaError_t launch_lse_merge(const float* part_o, const float* part_lse, int nsplit,
+                             __nv_bfloat16* o, float* lse, int B, int T, int Hq, int D,
+                             cudaStream_t stream) {
+  const long long rows = static_cast<long long>(B) * Hq * T;
+  if (rows == 0) return cudaSuccess;
+  const int threads = 256;
+  const unsigned blocks = static_cast<unsigned>((rows * 32 + threads - 1) / threads);
+  if (D == 128)
+    lse_merge_kernel<128><<<blocks, threads, 0, stream>>>(part_o, part_lse, nsplit, o, lse, B, T,
+                                                          Hq);
+  else
+    lse_merge_kernel<64><<<blocks, threads, 0, stream>>>(part_o, part_lse, nsplit, o, lse, B, T,
+                                                         Hq);
+  return cudaGetLastError();
+}
+
+// Device evaluation of the Phase-1 index math for every context row.
+__global__ void debug_index_kernel(int L, int b, int a, int32_t* blk, int32_t* pos,
+                                   int32_t* ranges) {
+  int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r >= L) return;
+  int out[4];
+  phase1_row_ranges(r, b, a, out);
+  blk[r] = r / b;
+  pos[r] = r;  // tokens keep their original global position IDs
+#pragma unroll
+  for (int j = 0; j < 4; ++j) ranges[4 * r + j] = out[j];
+}
+
+cudaError_t launch_debug_index(int L, int b, int a, int32_t* blk, int32_t* pos, int32_t* ranges,
+                               cudaStream_t stream) {
+  if (L <= 0) return cudaSuccess;
+  debug_index_kernel<<<ceil_div(L, 256), 256, 0, stream>>>(L, b, a, blk, pos, ranges);
+  return cudaGetLastError();
+}
+
+}  // namespace star

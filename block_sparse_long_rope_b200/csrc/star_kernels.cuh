@@ -1,0 +1,85 @@
+// Parameter blocks and launchers of the Star Attention kernels (internal to
+// the library; the public surface is include/star.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "star_index.cuh"
+
+namespace star {
+
+// ---- RoPE / cache write ----------------------------------------------------
+struct RopeJob {
+  const __nv_bfloat16* x;
+  __nv_bfloat16* y;
+  long long xs[3];  // element strides of (B, S, H); D is contiguous
+  long long ys[3];
+  int H;
+  int rotate;       // 0: plain copy (V into the cache)
+};
+struct RopeParams {
+  RopeJob job[3];
+  int B, S, D;
+  const int32_t* pos;  // nullable: position of token s is pos0 + s
+  long long pos0;
+  double inv_freq[64];  // theta^(-2i/D), i < D/2 (fp64, from the host)
+};
+// Fills p.inv_freq for head dim D and base theta.
+void rope_set_freq(RopeParams& p, int D, double theta);
+cudaError_t launch_rope(const RopeParams& p, int njobs, cudaStream_t stream);
+
+// ---- tcgen05 attention (Phase 1, and Phase 2 query chunks) -----------------
+struct AttnParams {
+  CUtensorMap tmQ;  // rotated Q [B, rows, Hq, D]: dims {D, Hq, rows, B}, box {64, 1, 128, 1}
+  CUtensorMap tmK;  // K cache [B*Hkv, Lvalid, D]: dims {D, Lvalid, B*Hkv}, box {64, 128, 1}
+  CUtensorMap tmV;  // V cache, same shape as K
+  AttnGeom geom;
+  int mode;         // 0: Phase 1 (bf16 o, lse), 1: Phase 2 partials
+  int num_items;
+  int qrows;        // rows per (batch, head) in the rotated-Q buffer
+  int nsplit;
+  __nv_bfloat16* o;  // Phase 1: [B, L, Hq, D]
+  float* lse;        // Phase 1: [B, Hq, L] (nullable)
+  float* part_o;     // Phase 2: [B, Hq, nsplit, T, D]
+  float* part_lse;   // Phase 2: [B, Hq, nsplit, T]
+  int* status;
+  float scale_log2;  // log2(e) / sqrt(D)
+  float scale_ln;    // 1 / sqrt(D)
+};
+size_t attn_smem_bytes(int D);
+cudaError_t launch_attn(const AttnParams& p, int D, cudaStream_t stream);
+
+// ---- Phase 2 decode (split-KV, HBM-bound) ----------------------------------
+constexpr int kDecRows = 16;   // (token, head) rows per CTA: one mma.sync M tile
+constexpr int kDecTile = 64;   // keys per staged K/V tile
+struct DecodeParams {
+  CUtensorMap tmK;  // K cache: dims {D, Lvalid, B*Hkv}, box {64, 64, 1}
+  CUtensorMap tmV;
+  const __nv_bfloat16* q;  // rotated q [B, T, Hq, D]
+  int B, T, Hq, Hkv, g, R;  // R = T * g rows (<= kDecRows)
+  int L, b, n, tail_len;    // context, block length, context splits, earlier tail tokens
+  int chunk;                // keys per CTA (multiple of kDecTile)
+  int nc_full, nc_last, nc_tail, chunks_per_head;  // chunk counts per split kind
+  float* ws_o;     // [B*Hkv, chunks_per_head, kDecRows, D] chunk-normalised output
+  float* ws_lse;   // [B*Hkv, chunks_per_head, kDecRows]
+  float* part_o;   // [B, Hq, n+1, T, D]
+  float* part_lse; // [B, Hq, n+1, T]
+  int* status;
+  float scale_log2, scale_ln;
+};
+size_t decode_smem_bytes(int D);
+cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t stream);
+
+// ---- LSE merge ---------------------------------------------------------------
+cudaError_t launch_lse_merge(const float* part_o, const float* part_lse, int nsplit,
+                             __nv_bfloat16* o, float* lse, int B, int T, int Hq, int D,
+                             cudaStream_t stream);
+
+// ---- debug: device-evaluated index math --------------------------------------
+cudaError_t launch_debug_index(int L, int b, int a, int32_t* blk, int32_t* pos, int32_t* ranges,
+                               cudaStream_t stream);
+
+}  // namespace star

@@ -1,0 +1,135 @@
+"""Python binding of the C ABI (include/star.h), same names, torch tensors in.
+
+Only argument marshalling happens here: pointers, sizes and the current CUDA
+stream are passed to libstar.so, which validates and launches. PyTorch serves
+for device memory and streams.
+"""
+import ctypes
+
+import torch
+
+from . import _abi
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _bf16(t, name):
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name} must be bfloat16, got {t.dtype}")
+
+
+def _i64x3(vals):
+    return (ctypes.c_int64 * 3)(*[int(v) for v in vals])
+
+
+def version() -> str:
+    return _abi.load().star_version().decode()
+
+
+def star_rope(x, y, theta, pos=None, pos0=0, stream=None):
+    """y[b,s,h,:] = RoPE(x[b,s,h,:]) at position pos[s] (or pos0 + s).
+    x, y: bf16 [B, S, H, D] views (any strides with D contiguous)."""
+    _bf16(x, "x")
+    _bf16(y, "y")
+    B, S, H, D = x.shape
+    if tuple(y.shape) != (B, S, H, D):
+        raise ValueError("x and y shapes differ")
+    if x.stride(3) != 1 or y.stride(3) != 1:
+        raise ValueError("head_dim must be contiguous")
+    if pos is not None and pos.dtype != torch.int32:
+        raise TypeError("pos must be int32")
+    lib = _abi.load()
+    _abi.check(lib.star_rope(_ptr(x), _i64x3(x.stride()[:3]), _ptr(y), _i64x3(y.stride()[:3]),
+                             _ptr(pos), int(pos0), B, S, H, D, float(theta), _stream(stream)))
+    return y
+
+
+def star_phase1_workspace_bytes(B, L, Hq, D) -> int:
+    return int(_abi.load().star_phase1_workspace_bytes(B, L, Hq, D))
+
+
+def star_phase1_encode(q, k, v, o, k_cache, v_cache, block_len, anchor_len, theta, workspace,
+                       lse=None, stream=None):
+    """Phase 1: q[B,L,Hq,D], k/v[B,L,Hkv,D] (pre-RoPE bf16) -> o[B,L,Hq,D] bf16,
+    cache rows [0,L) of k_cache/v_cache[B,Hkv,Lcap,D], lse[B,Hq,L] fp32 (optional)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _bf16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    Lcap = k_cache.shape[2]
+    if lse is not None and (lse.dtype != torch.float32 or not lse.is_contiguous()):
+        raise ValueError("lse must be contiguous float32")
+    lib = _abi.load()
+    _abi.check(lib.star_phase1_encode(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(k_cache), _ptr(v_cache), Lcap, _ptr(lse), B, L,
+        Hq, Hkv, D, int(block_len), int(anchor_len), float(theta), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o
+
+
+def star_phase2_workspace_bytes(B, T, Hq, Hkv, D, Lcap, block_len) -> int:
+    return int(_abi.load().star_phase2_workspace_bytes(B, T, Hq, Hkv, D, Lcap, block_len))
+
+
+def star_phase2_partial(q, k, v, k_cache, v_cache, L, block_len, tail_len, part_o, part_lse,
+                        theta, workspace, stream=None):
+    """Phase 2 partials for T new tokens (q[B,T,Hq,D], k/v[B,T,Hkv,D] pre-RoPE)
+    at positions L + tail_len + t. Appends k/v to the cache; writes
+    part_o[B,Hq,n+1,T,D], part_lse[B,Hq,n+1,T]. Returns nsplit = n + 1."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _bf16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    Lcap = k_cache.shape[2]
+    ns = ctypes.c_int(0)
+    lib = _abi.load()
+    _abi.check(lib.star_phase2_partial(
+        _ptr(q), _ptr(k), _ptr(v), T, _ptr(k_cache), _ptr(v_cache), Lcap, int(L), int(block_len),
+        int(tail_len), _ptr(part_o), _ptr(part_lse), ctypes.byref(ns), B, Hq, Hkv, D,
+        float(theta), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return ns.value
+
+
+def star_lse_merge(part_o, part_lse, o, lse=None, stream=None):
+    """Exact merge: part_o[B,Hq,S,T,D], part_lse[B,Hq,S,T] -> o[B,T,Hq,D] bf16, lse[B,Hq,T]."""
+    B, Hq, S, T, D = part_o.shape
+    _bf16(o, "o")
+    lib = _abi.load()
+    _abi.check(lib.star_lse_merge(_ptr(part_o), _ptr(part_lse), S, _ptr(o), _ptr(lse), B, T, Hq,
+                                  D, _stream(stream)))
+    return o
+
+
+def star_device_status(workspace, stream=None):
+    """Synchronise, read and clear the device status word; raises on a device error."""
+    lib = _abi.load()
+    _abi.check(lib.star_device_status(_ptr(workspace), _stream(stream)))
+
+
+def star_debug_index(L, block_len, anchor_len, device="cuda", stream=None):
+    """Device-evaluated index math: (blk[L], pos[L], kv_ranges[L,4]) int32."""
+    blk = torch.empty(L, dtype=torch.int32, device=device)
+    pos = torch.empty(L, dtype=torch.int32, device=device)
+    rng = torch.empty((L, 4), dtype=torch.int32, device=device)
+    lib = _abi.load()
+    _abi.check(lib.star_debug_index(L, block_len, anchor_len, _ptr(blk), _ptr(pos), _ptr(rng),
+                                    _stream(stream)))
+    return blk, pos, rng
+
+
+def alloc_workspace(nbytes, device="cuda"):
+    """A caller-owned workspace (the library itself allocates nothing)."""
+    n = max(256, (int(nbytes) + 255) // 256 * 256)
+    return torch.empty(n, dtype=torch.uint8, device=device)

@@ -1,0 +1,182 @@
+/*
+ * star.h — C ABI of the Star Attention hot path for NVIDIA B200 (sm_100a).
+ *
+ * Star Attention (arXiv 2411.17116) encodes a long context in two phases:
+ *   Phase 1  the context is split into blocks c_1..c_n of b tokens; every
+ *            block i >= 2 is prefixed with the anchor block c_1, which keeps
+ *            its original position IDs, and attends causally only inside that
+ *            augmented block; the anchor's KV entries are then dropped
+ *            [pith 2WVXFXZ2, "What carries the argument"; minor comment on
+ *            Section 2.1: c'_1 = c_1 has b tokens, only blocks i >= 2 carry
+ *            the anchor].
+ *   Phase 2  query and generated tokens attend to every cached token: each
+ *            block ("host") returns a local attention output and a softmax
+ *            statistic, and the query side re-weights them into exact
+ *            global attention [pith 2WVXFXZ2, Referee summary; Circularity
+ *            check; minor comment on Algorithm 2: weight exp(s_h - s_global)].
+ * On one GPU the pages' hosts become blocks processed in parallel.
+ *
+ * Conventions shared by every call
+ *   - Memory is owned by the caller (device pointers unless stated). The
+ *     library allocates nothing and keeps no state besides a thread-local
+ *     error message and per-device properties it caches on first use.
+ *   - Every call is asynchronous on `cuda_stream` (a cudaStream_t; NULL is
+ *     the legacy default stream). None synchronises, except
+ *     star_device_status.
+ *   - Arguments are validated before anything is launched; on a non-OK
+ *     status nothing was enqueued (except STAR_ERR_CUDA from a launch).
+ *   - Element types: bf16 for Q/K/V/O and the KV cache, fp32 for LSE and
+ *     partials. LSE values are natural logarithms.
+ *   - Softmax scale 1/sqrt(D). Query head h uses KV head h / (Hq / Hkv)
+ *     (contiguous GQA groups).
+ *   - RoPE is rotate-half with base theta: pair (x_i, x_{i+D/2}) turns by the
+ *     angle p * theta^(-2i/D); token t of the context sits at position t, so
+ *     the anchor keeps positions 0..a-1 in every block.
+ *   - Supported head_dim D: 64 and 128. Pointers must be 16-byte aligned.
+ *   - Device errors found inside kernels (a bounded wait that gave up, an
+ *     index outside its buffer) are recorded in a status word at the start of
+ *     the call's workspace and read back by star_device_status.
+ */
+#ifndef STAR_H_
+#define STAR_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  STAR_OK = 0,
+  STAR_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size or shape */
+  STAR_ERR_UNSUPPORTED = 2,   /* head_dim or device not supported */
+  STAR_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed */
+  STAR_ERR_DEVICE_TIMEOUT = 4,/* a kernel's bounded wait gave up */
+  STAR_ERR_DEVICE_BOUNDS = 5  /* a kernel found an index outside its buffer */
+} star_status;
+
+/* Message describing the calling thread's last non-OK status ("" if none).
+ * The pointer stays valid until the next call on the same thread. */
+const char* star_last_error(void);
+
+/* Library version string. */
+const char* star_version(void);
+
+/*
+ * star_rope — rotate-half RoPE at given positions
+ * [pith 2607.20457, "What carries the argument": original global position
+ * IDs preserve RoPE distances; pith 2WVXFXZ2: the anchor keeps c_1's
+ * original positional indices].
+ *
+ *   y[b,s,h,:] = RoPE(x[b,s,h,:], p_s),  p_s = pos[s] if pos != NULL else pos0 + s
+ *
+ * x, y: bf16, D contiguous; x_stride / y_stride give the element strides of
+ * the (B, S, H) dimensions (each a multiple of 8). x and y may be the same
+ * buffer (in place) but must not otherwise overlap. pos: device int32[S] or
+ * NULL. The angle p * theta_i is formed and reduced modulo 2*pi in fp64;
+ * sine/cosine and the rotation run in fp32; y is rounded to bf16 (nearest
+ * even).
+ */
+star_status star_rope(const void* x, const int64_t x_stride[3], void* y,
+                      const int64_t y_stride[3], const int32_t* pos, int64_t pos0, int B,
+                      int S, int H, int D, double theta, void* cuda_stream);
+
+/* Workspace bytes star_phase1_encode needs: the rotated Q (bf16
+ * [B, L, Hq, D]) plus a 256-byte status header. */
+size_t star_phase1_workspace_bytes(int B, int L, int Hq, int D);
+
+/*
+ * star_phase1_encode — Phase 1, anchor-block blockwise-local causal encoding
+ * [pith 2WVXFXZ2, "What carries the argument"; minor comment on
+ * Section 2.1; abstract: "the context is processed using blockwise-local
+ * attention ... in parallel"].
+ *
+ * Inputs (pre-RoPE, token-major): q[B, L, Hq, D], k/v[B, L, Hkv, D].
+ * Row r of block i = r / block_len attends to
+ *   i == 0 : keys [0, r]                       (c'_1 = c_1, plain causal)
+ *   i >= 1 : keys [0, anchor_len) U [i*block_len, r]
+ * The anchor's keys are block 1's cache rows (same tokens, same positions),
+ * so they are computed once and shared; no anchor copy is ever stored.
+ * Outputs:
+ *   o[B, L, Hq, D]             bf16, softmax-normalised
+ *   k_cache/v_cache[B, Hkv, Lcap, D]  rows [0, L) written: K rotated, V copied
+ *                              (head-major; rows >= L untouched)
+ *   lse[B, Hq, L]              fp32 natural-log statistic, or NULL
+ * anchor_len in [0, block_len]; 0 disables the anchor (the pages' "no
+ * anchor" ablation); block_len >= L gives full causal attention.
+ * Requires Lcap >= L, workspace_bytes >= star_phase1_workspace_bytes().
+ */
+star_status star_phase1_encode(const void* q, const void* k, const void* v, void* o,
+                               void* k_cache, void* v_cache, int Lcap, float* lse, int B, int L,
+                               int Hq, int Hkv, int D, int block_len, int anchor_len,
+                               double theta, void* workspace, size_t workspace_bytes,
+                               void* cuda_stream);
+
+/* Workspace bytes star_phase2_partial needs for up to T new tokens with a
+ * cache of capacity Lcap (context L plus tail) split into blocks of
+ * block_len. */
+size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lcap, int block_len);
+
+/*
+ * star_phase2_partial — Phase 2 per-block partial attention
+ * [pith 2WVXFXZ2, Referee summary: the query is broadcast and each host
+ * computes local softmax statistics; abstract: query and response tokens
+ * attend to all prior cached tokens].
+ *
+ * T new tokens (a query chunk, or one decode token) with pre-RoPE
+ * q[B, T, Hq, D], k/v[B, T, Hkv, D] sit at positions L + tail_len + t. The
+ * call rotates q and k, appends k/v into cache rows L + tail_len + t, then
+ * for every split writes the split-local softmax-normalised output and its
+ * LSE:
+ *   split j < n (n = ceil(L / block_len)): context block j, keys
+ *                 [j*block_len, min((j+1)*block_len, L)), all visible
+ *   split n (tail): cache rows [L, L + tail_len + t], causal per token
+ *   part_o[B, Hq, n+1, T, D] fp32, part_lse[B, Hq, n+1, T] fp32
+ * *nsplit_out (host int, may be NULL) receives n + 1.
+ * Requires Lcap >= L + tail_len + T and cache rows [0, L + tail_len) filled
+ * by earlier calls; workspace_bytes >= star_phase2_workspace_bytes().
+ */
+star_status star_phase2_partial(const void* q, const void* k, const void* v, int T, void* k_cache,
+                                void* v_cache, int Lcap, int L, int block_len, int tail_len,
+                                float* part_o, float* part_lse, int* nsplit_out, int B, int Hq,
+                                int Hkv, int D, double theta, void* workspace,
+                                size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * star_lse_merge — exact merge of per-split partials into global attention
+ * [pith 2WVXFXZ2, minor comment on Algorithm 2 (corrected update
+ * exp(s_h - s_global) * A_h); assumptions: online softmax aggregation gives
+ * the exact global softmax]:
+ *   m = max_h lse_h,  w_h = exp(lse_h - m),
+ *   o = sum_h w_h o_h / sum_h w_h   -> o[B, T, Hq, D] bf16
+ *   lse = m + log(sum_h w_h)        -> lse[B, Hq, T] fp32 (NULL to skip)
+ * Splits whose lse is -inf carry weight 0. Inputs as star_phase2_partial
+ * writes them.
+ */
+star_status star_lse_merge(const float* part_o, const float* part_lse, int nsplit, void* o,
+                           float* lse, int B, int T, int Hq, int D, void* cuda_stream);
+
+/*
+ * star_device_status — synchronises `cuda_stream`, then reads and clears the
+ * status word at the start of `workspace` (a workspace passed to
+ * star_phase1_encode or star_phase2_partial). Returns STAR_OK,
+ * STAR_ERR_DEVICE_TIMEOUT or STAR_ERR_DEVICE_BOUNDS (message in
+ * star_last_error), or STAR_ERR_CUDA.
+ */
+star_status star_device_status(void* workspace, void* cuda_stream);
+
+/*
+ * star_debug_index — evaluates the kernels' index math on the device for
+ * every context row r in [0, L): blk[r] = block id, pos[r] = position ID,
+ * kv_ranges[4r..4r+3] = {anchor_lo, anchor_hi, own_lo, own_hi} (half-open;
+ * block 0 reports an empty anchor range [0, 0)). Device int32 outputs.
+ */
+star_status star_debug_index(int L, int block_len, int anchor_len, int32_t* blk, int32_t* pos,
+                             int32_t* kv_ranges, void* cuda_stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STAR_H_ */

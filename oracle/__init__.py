@@ -10,6 +10,7 @@ from .oracle import (  # noqa: F401
     phase1_full,
     phase1_ranges,
     phase1_rows,
+    phase1_rows_selected,
     phase2_rows,
     rope,
     round_bf16,

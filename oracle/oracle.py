@@ -30,6 +30,9 @@ def _load():
             lib.orc_phase1_rows.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                             ctypes.c_double, ctypes.c_int, _I, _P, _P, _P,
                                             _P, _P, _P]
+            lib.orc_phase1_rows_sel.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                                ctypes.c_double, ctypes.c_int, _I, _P, _P, _P,
+                                                _P, _P, _P]
             lib.orc_phase2_rows.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                             _I, _I, ctypes.c_double, ctypes.c_int, _I, _P,
                                             _P, _P, _P, _P]
@@ -38,6 +41,7 @@ def _load():
                                             _P, _P, _P]
             lib.orc_lse_merge.argtypes = [_P, _P, _I, _I, _I, _P, _P]
             for f in ("orc_round_bf16", "orc_rope", "orc_phase1_ranges", "orc_phase1_rows",
+                      "orc_phase1_rows_sel",
                       "orc_phase2_rows", "orc_global_rows", "orc_lse_merge"):
                 getattr(lib, f).restype = None
             _lib = lib
@@ -100,6 +104,26 @@ def phase1_rows(q, k, v, block_len, anchor_len, theta, qb, qh, qr, round_qk=True
     _load().orc_phase1_rows(_ptr(qbits), _ptr(kbits), _ptr(vbits), B, L, Hq, Hkv, D, block_len,
                             anchor_len, float(theta), int(bool(round_qk)), nq, _ptr(qb), _ptr(qh),
                             _ptr(qr), _ptr(o), _ptr(lse), _ptr(nvis))
+    return o, lse, nvis
+
+
+def phase1_rows_selected(q_sel, k, v, block_len, anchor_len, theta, qb, qh, qr, Hq,
+                         round_qk=True):
+    """As phase1_rows, with q_sel[nq, D] (bf16) holding only the listed queries'
+    pre-RoPE vectors (for contexts too long to copy Q to the host whole)."""
+    qbits, kbits, vbits = bf16_bits(q_sel), bf16_bits(k), bf16_bits(v)
+    B, L, Hkv, D = kbits.shape
+    qb = np.ascontiguousarray(qb, dtype=np.int64)
+    qh = np.ascontiguousarray(qh, dtype=np.int64)
+    qr = np.ascontiguousarray(qr, dtype=np.int64)
+    nq = qb.size
+    assert qbits.shape == (nq, D)
+    o = np.empty((nq, D), dtype=np.float64)
+    lse = np.empty((nq,), dtype=np.float64)
+    nvis = np.empty((nq,), dtype=np.int64)
+    _load().orc_phase1_rows_sel(_ptr(qbits), _ptr(kbits), _ptr(vbits), L, Hq, Hkv, D, block_len,
+                                anchor_len, float(theta), int(bool(round_qk)), nq, _ptr(qb),
+                                _ptr(qh), _ptr(qr), _ptr(o), _ptr(lse), _ptr(nvis))
     return o, lse, nvis
 
 

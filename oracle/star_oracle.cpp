@@ -218,10 +218,11 @@ void orc_phase1_ranges(i64 L, i64 block_len, i64 anchor_len, i64* blk, i64* rang
 // positions 0..a-1). If round_qk, rotated Q and K are rounded to bf16 (the
 // precision the rotated tensors and the KV cache are stored in).
 // Outputs: o[nq, D], lse[nq] (natural log), nvis[nq] (nullable).
-void orc_phase1_rows(const uint16_t* q_bits, const uint16_t* k_bits, const uint16_t* v_bits, i64 B,
-                     i64 L, i64 Hq, i64 Hkv, i64 D, i64 block_len, i64 anchor_len, double theta,
-                     int round_qk, i64 nq, const i64* qb, const i64* qh, const i64* qr, double* o,
-                     double* lse, i64* nvis) {
+// q_sel != 0 means q_bits holds only the listed queries' vectors, [nq, D].
+static void phase1_rows_impl(const uint16_t* q_bits, int q_sel, const uint16_t* k_bits,
+                             const uint16_t* v_bits, i64 L, i64 Hq, i64 Hkv, i64 D, i64 block_len,
+                             i64 anchor_len, double theta, int round_qk, i64 nq, const i64* qb,
+                             const i64* qh, const i64* qr, double* o, double* lse, i64* nvis) {
   const i64 g = Hq / Hkv;
   const double scale = 1.0 / std::sqrt(static_cast<double>(D));
   // Group queries by (batch, kv head) so each group's keys are rotated once.
@@ -238,7 +239,7 @@ void orc_phase1_rows(const uint16_t* q_bits, const uint16_t* k_bits, const uint1
     for (size_t j = 0; j < qs.size(); ++j) {
       i64 i = qs[j];
       std::vector<double> x(D), q(D);
-      const uint16_t* src = q_bits + ((b * L + qr[i]) * Hq + qh[i]) * D;
+      const uint16_t* src = q_sel ? q_bits + i * D : q_bits + ((b * L + qr[i]) * Hq + qh[i]) * D;
       for (i64 d = 0; d < D; ++d) x[d] = bf16_to_double(src[d]);
       rope_vec(x.data(), q.data(), D, static_cast<double>(qr[i]), theta);
       if (round_qk)
@@ -249,6 +250,24 @@ void orc_phase1_rows(const uint16_t* q_bits, const uint16_t* k_bits, const uint1
           [&](i64 c) { return V.data() + c * D; }, o + i * D, lse + i, nvis ? nvis + i : nullptr);
     }
   }
+}
+
+void orc_phase1_rows(const uint16_t* q_bits, const uint16_t* k_bits, const uint16_t* v_bits, i64 B,
+                     i64 L, i64 Hq, i64 Hkv, i64 D, i64 block_len, i64 anchor_len, double theta,
+                     int round_qk, i64 nq, const i64* qb, const i64* qh, const i64* qr, double* o,
+                     double* lse, i64* nvis) {
+  (void)B;
+  phase1_rows_impl(q_bits, 0, k_bits, v_bits, L, Hq, Hkv, D, block_len, anchor_len, theta,
+                   round_qk, nq, qb, qh, qr, o, lse, nvis);
+}
+
+// As orc_phase1_rows, with q_sel_bits[nq, D] holding only the listed queries.
+void orc_phase1_rows_sel(const uint16_t* q_sel_bits, const uint16_t* k_bits,
+                         const uint16_t* v_bits, i64 L, i64 Hq, i64 Hkv, i64 D, i64 block_len,
+                         i64 anchor_len, double theta, int round_qk, i64 nq, const i64* qb,
+                         const i64* qh, const i64* qr, double* o, double* lse, i64* nvis) {
+  phase1_rows_impl(q_sel_bits, 1, k_bits, v_bits, L, Hq, Hkv, D, block_len, anchor_len, theta,
+                   round_qk, nq, qb, qh, qr, o, lse, nvis);
 }
 
 // Phase 2 partials ([pith 2WVXFXZ2, Referee summary and Circularity check]):

@@ -1,0 +1,113 @@
+"""GPU parity of Phase 2 (star_phase2_partial + star_lse_merge) against the
+fp64 oracle: per-split partials, the merged output, and equality with one-shot
+global attention over every cached key. Covers the tensor-core query-chunk
+path (T*g > 16) and the split-KV decode path (T*g <= 16), ragged blocks, and
+a tail that grows across calls."""
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_long_rope_b200 import build as star_build
+from block_sparse_long_rope_b200 import star
+from oracle import oracle as orc
+
+from gpu_util import TOL_LSE, TOL_O, max_abs, rand_bf16, to64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    star_build.build()
+    torch.cuda.init()
+
+
+def run_flow(B, L, Hq, Hkv, D, b, a, theta, Ts, seed):
+    """Encode the context, then Phase-2 calls of sizes Ts in order; check every
+    call's partials and merged output against the oracle."""
+    dev = "cuda"
+    q = rand_bf16((B, L, Hq, D), seed=seed)
+    k = rand_bf16((B, L, Hkv, D), seed=seed + 1)
+    v = rand_bf16((B, L, Hkv, D), seed=seed + 2)
+    Ttot = sum(Ts)
+    Lcap = L + Ttot + 5
+    kc = torch.full((B, Hkv, Lcap, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    vc = torch.full((B, Hkv, Lcap, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    o = torch.empty_like(q)
+    ws1 = star.alloc_workspace(star.star_phase1_workspace_bytes(B, L, Hq, D))
+    star.star_phase1_encode(q, k, v, o, kc, vc, b, a, theta, ws1)
+    star.star_device_status(ws1)
+    n = -(-L // b)
+    qn = rand_bf16((B, Ttot, Hq, D), seed=seed + 3)
+    kn = rand_bf16((B, Ttot, Hkv, D), seed=seed + 4)
+    vn = rand_bf16((B, Ttot, Hkv, D), seed=seed + 5)
+    tail = 0
+    for T in Ts:
+        qt = qn[:, tail:tail + T].contiguous()
+        kt = kn[:, tail:tail + T].contiguous()
+        vt = vn[:, tail:tail + T].contiguous()
+        po = torch.full((B, Hq, n + 1, T, D), float("nan"), device=dev)
+        pl = torch.full((B, Hq, n + 1, T), float("nan"), device=dev)
+        ws = star.alloc_workspace(star.star_phase2_workspace_bytes(B, T, Hq, Hkv, D, Lcap, b))
+        ns = star.star_phase2_partial(qt, kt, vt, kc, vc, L, b, tail, po, pl, theta, ws)
+        assert ns == n + 1
+        om = torch.empty((B, T, Hq, D), dtype=torch.bfloat16, device=dev)
+        lm = torch.empty((B, Hq, T), device=dev)
+        star.star_lse_merge(po, pl, om, lm)
+        star.star_device_status(ws)
+        torch.cuda.synchronize()
+        bb, hh, tt = np.meshgrid(np.arange(B), np.arange(Hq), np.arange(T), indexing="ij")
+        bb, hh, tt = bb.ravel(), hh.ravel(), tt.ravel()
+        # the oracle sees the raw context and every tail token so far
+        kt_all, vt_all = kn[:, : tail + T].cpu(), vn[:, : tail + T].cpu()
+        rpo, rpl = [], []
+        for bi in range(B):  # the oracle's tail tensors are per batch row
+            sel = bb == bi
+            o_, l_ = orc.phase2_rows(qt[bi:bi + 1].cpu(), k[bi:bi + 1].cpu(), v[bi:bi + 1].cpu(),
+                                     kt_all[bi:bi + 1], vt_all[bi:bi + 1], b, tail, theta,
+                                     np.zeros(sel.sum()), hh[sel], tt[sel])
+            rpo.append(o_)
+            rpl.append(l_)
+        rpo = np.concatenate(rpo)
+        rpl = np.concatenate(rpl)
+        gpo = to64(po).transpose(0, 1, 3, 2, 4).reshape(-1, n + 1, D)
+        gpl = to64(pl).transpose(0, 1, 3, 2).reshape(-1, n + 1)
+        assert max_abs(gpo, rpo) <= TOL_O, f"T={T} tail={tail}"
+        assert max_abs(gpl, rpl) <= TOL_LSE, f"T={T} tail={tail}"
+        mo, ml = orc.lse_merge(rpo, rpl)
+        go = to64(om).transpose(0, 2, 1, 3).reshape(-1, D)
+        gl = to64(lm).reshape(-1)
+        assert max_abs(go, mo) <= TOL_O
+        assert max_abs(gl, ml) <= TOL_LSE
+        # exactness of the merge: equals one-shot attention over all cached keys
+        go2, gl2 = [], []
+        for bi in range(B):
+            sel = bb == bi
+            o_, l_ = orc.global_rows(qt[bi:bi + 1].cpu(), k[bi:bi + 1].cpu(), v[bi:bi + 1].cpu(),
+                                     kt_all[bi:bi + 1], vt_all[bi:bi + 1], tail, theta,
+                                     np.zeros(sel.sum()), hh[sel], tt[sel])
+            go2.append(o_)
+            gl2.append(l_)
+        assert max_abs(go, np.concatenate(go2)) <= TOL_O
+        assert max_abs(gl, np.concatenate(gl2)) <= TOL_LSE
+        # the appended cache rows hold the rotated new keys
+        kref = orc.rope(kt.cpu(), np.arange(L + tail, L + tail + T), theta, round_out=True)
+        kgot = to64(kc[:, :, L + tail:L + tail + T]).transpose(0, 2, 1, 3)
+        np.testing.assert_array_equal(kgot, kref)  # correctly rounded: bit-exact
+        tail += T
+
+
+# (B, L, Hq, Hkv, D, b, a, theta, Ts)
+FLOWS = [
+    (1, 2048, 4, 1, 64, 512, 512, 1e4, [16, 1, 1, 1, 1, 1, 1, 1, 1]),  # tiny: 16 + 8 decode
+    (2, 1000, 4, 2, 64, 300, 100, 1e4, [5, 20, 1, 1, 1]),             # R=10 decode, then chunk
+    (1, 700, 16, 2, 128, 256, 256, 5e5, [2, 3, 1, 1]),                # g=8: R=16 decode, R=24 chunk
+    (1, 900, 2, 2, 128, 200, 200, 5e5, [1, 130, 1]),                  # g=1: T=130 = 2 query tiles
+    (1, 4096, 32, 8, 128, 1024, 1024, 5e5, [128, 1, 1]),              # 8B layer shape, short context
+]
+
+
+@pytest.mark.parametrize("flow", FLOWS, ids=[f"L{f[1]}b{f[5]}g{f[2]//f[3]}D{f[4]}T{'-'.join(map(str, f[8]))}" for f in FLOWS])
+def test_phase2_flow_matches_oracle(flow):
+    B, L, Hq, Hkv, D, b, a, theta, Ts = flow
+    run_flow(B, L, Hq, Hkv, D, b, a, theta, Ts, seed=L)
