@@ -13,7 +13,7 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libstar.so")
 OBJ_DIR = os.path.join(HERE, "_build")
 
-SOURCES = ["api.cu", "rope.cu", "lse_merge.cu", "phase2_decode.cu", "phase1_sm100.cu"]
+SOURCES = ["api.cu", "rope.cu", "lse_merge.cu", "phase2_decode.cu", "phase1_sm100.cu", "noalloc.cu"]
 HEADERS = ["star_common.cuh", "star_index.cuh", "star_kernels.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

@@ -172,6 +172,12 @@ size_t decode_scratch_bytes(int B, int Hkv, int D, int Lcap, int block_len) {
 
 }  // namespace
 
+namespace star {
+// Sets the calling thread's message for star_last_error (used by entry points
+// defined in other files of the library).
+void set_last_error(const char* msg) { g_err = msg; }
+}  // namespace star
+
 extern "C" {
 
 const char* star_last_error(void) { return g_err.c_str(); }

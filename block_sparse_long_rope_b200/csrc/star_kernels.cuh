@@ -78,6 +78,9 @@ cudaError_t launch_lse_merge(const float* part_o, const float* part_lse, int nsp
                              __nv_bfloat16* o, float* lse, int B, int T, int Hq, int D,
                              cudaStream_t stream);
 
+// ---- error message of the calling thread (star_last_error) -------------------
+void set_last_error(const char* msg);
+
 // ---- debug: device-evaluated index math --------------------------------------
 cudaError_t launch_debug_index(int L, int b, int a, int32_t* blk, int32_t* pos, int32_t* ranges,
                                cudaStream_t stream);

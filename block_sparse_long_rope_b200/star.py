@@ -102,6 +102,26 @@ def star_phase2_partial(q, k, v, k_cache, v_cache, L, block_len, tail_len, part_
     return ns.value
 
 
+def star_phase2_decode_static(q, k, v, k_cache, v_cache, L, block_len, tail_len, part_o,
+                              part_lse, theta, stream=None):
+    """star_phase2_partial for decode steps without a workspace: the scratch
+    lives in the library's fixed 16 MiB device array (see include/star.h)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _bf16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    Lcap = k_cache.shape[2]
+    ns = ctypes.c_int(0)
+    lib = _abi.load()
+    _abi.check(lib.star_phase2_decode_static(
+        _ptr(q), _ptr(k), _ptr(v), T, _ptr(k_cache), _ptr(v_cache), Lcap, int(L), int(block_len),
+        int(tail_len), _ptr(part_o), _ptr(part_lse), ctypes.byref(ns), B, Hq, Hkv, D,
+        float(theta), _stream(stream)))
+    return ns.value
+
+
 def star_lse_merge(part_o, part_lse, o, lse=None, stream=None):
     """Exact merge: part_o[B,Hq,S,T,D], part_lse[B,Hq,S,T] -> o[B,T,Hq,D] bf16, lse[B,Hq,T]."""
     B, Hq, S, T, D = part_o.shape

@@ -158,6 +158,34 @@ star_status star_lse_merge(const float* part_o, const float* part_lse, int nspli
                            float* lse, int B, int T, int Hq, int D, void* cuda_stream);
 
 /*
+ * star_phase2_decode_static — star_phase2_partial for decode steps
+ * (T * (Hq / Hkv) <= 16) without a workspace argument. The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory themselves, such as a plugin whose host application owns
+ * every device allocation, or a serving loop that must never block in
+ * cudaMalloc/cudaFree. Its scratch (the rotated query and the per-chunk
+ * partials) lives in a 16 MiB device array inside the library, which every
+ * GPU that loads the library keeps until the process exits; the caller still
+ * passes inputs and outputs, with the same meaning and layout as
+ * star_phase2_partial.
+ *   - The array's address is looked up once per device on the first call made
+ *     with that device current; make that first call before any stream
+ *     capture.
+ *   - All calls on a device share the array, which keeps the previous call's
+ *     contents (the status word is cleared by each call; the rest is rewritten
+ *     before it is read). Calls whose work overlaps on the GPU race on it:
+ *     serialise them (one stream, or explicit ordering).
+ *   - Sizes whose scratch cannot fit 16 MiB even with the largest chunk, or
+ *     T * g > 16, return STAR_ERR_INVALID_ARG before anything is enqueued.
+ *     Nothing is allocated.
+ */
+star_status star_phase2_decode_static(const void* q, const void* k, const void* v, int T,
+                                      void* k_cache, void* v_cache, int Lcap, int L,
+                                      int block_len, int tail_len, float* part_o,
+                                      float* part_lse, int* nsplit_out, int B, int Hq, int Hkv,
+                                      int D, double theta, void* cuda_stream);
+
+/*
  * star_device_status — synchronises `cuda_stream`, then reads and clears the
  * status word at the start of `workspace` (a workspace passed to
  * star_phase1_encode or star_phase2_partial). Returns STAR_OK,
