@@ -136,6 +136,24 @@ def oracle_sample(w, budget_s=15.0, seed=0):
     return est_step, sample, t_p1 + t_dec
 
 
+def max_over_ranks(values, device, world):
+    """Element-wise max of per-rank timings (ms) over all ranks."""
+    if world <= 1:
+        return list(values)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor(list(values), device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def job_value(tokens_per_rank, world, ms_per_step):
+    """Whole-job throughput: tokens all ranks processed per second of the
+    slowest rank's step time."""
+    return tokens_per_rank * world / (ms_per_step / 1e3)
+
+
 def omp_threads():
     v = os.environ.get("OMP_NUM_THREADS")
     return int(v) if v else (os.cpu_count() or 1)
@@ -208,10 +226,8 @@ def run_star(args, w, rank, world, local_rank):
     star.star_device_status(layer.buf.ws1)
     star.star_device_status(layer.buf.ws2)
 
-    if world > 1:
-        t = torch.tensor([elapsed_ms, p1_ms, chunk_ms, dec_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed_ms, p1_ms, chunk_ms, dec_ms = t.tolist()
+    elapsed_ms, p1_ms, chunk_ms, dec_ms = max_over_ranks(
+        [elapsed_ms, p1_ms, chunk_ms, dec_ms], dev, world)
 
     # ---- end to end through the public API with host buffers ----------------
     host_ctx = [t.cpu().pin_memory() for t in ctx]
@@ -249,11 +265,7 @@ def run_star(args, w, rank, world, local_rank):
         e2e_step()
     e2.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = s2.elapsed_time(e2)
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
+    e2e_ms = max_over_ranks([s2.elapsed_time(e2)], dev, world)[0]
 
     if rank != 0:
         return None
@@ -261,7 +273,7 @@ def run_star(args, w, rank, world, local_rank):
     K = args.steps
     ms_step = elapsed_ms / K
     ctx_tokens = w.B * w.L * world
-    value = ctx_tokens / (ms_step / 1e3)
+    value = job_value(w.B * w.L, world, ms_step)
     p1_s = p1_ms / K / 1e3
     p1_flops = w.phase1_flops()
     p1_tflops = p1_flops / p1_s / 1e12
@@ -317,7 +329,7 @@ def run_star(args, w, rank, world, local_rank):
                      "algorithmic": "4*D*Hq*B*[n*b(b+1)/2 + (n-1)*a*b] unmasked FLOPs per launch "
                                     f"= {p1_flops:.4g}",
                      "traffic": None},
-        "e2e": {"value": round(ctx_tokens / (e2e_ms / K / 1e3), 1), "unit": "tok/s",
+        "e2e": {"value": round(job_value(w.B * w.L, world, e2e_ms / K), 1), "unit": "tok/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": launches * K,
         "clocks": clocks,
@@ -379,20 +391,21 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        # rank 0 alone times the oracle on the host cores; other ranks exit 0
+        line = run_reference(args, w, rank)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
     if world > 1:
         import datetime
 
         import torch
         import torch.distributed as dist
-        backend = "nccl" if args.impl == "star" else "gloo"
-        if backend == "nccl":
-            torch.cuda.set_device(local_rank)
-        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group(backend="nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        if args.impl == "reference":
-            line = run_reference(args, w, rank)
-        else:
-            line = run_star(args, w, rank, world, local_rank)
+        line = run_star(args, w, rank, world, local_rank)
         if rank == 0 and line is not None:
             print(json.dumps(line), flush=True)
     finally:

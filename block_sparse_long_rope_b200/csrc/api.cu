@@ -12,7 +12,7 @@
 #include <mutex>
 #include <string>
 
-#include "../../include/star.h"
+#include "star.h"
 #include "star_common.cuh"
 #include "star_kernels.cuh"
 

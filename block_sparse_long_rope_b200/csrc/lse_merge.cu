@@ -33,29 +33,40 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict_
   const int b = warp / (T * Hq);
   const size_t bh = static_cast<size_t>(b) * Hq + h;
 
+  // statistics: lanes read the split LSEs in parallel, shuffles reduce them
   float m = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) m = fmaxf(m, part_lse[(bh * nsplit + s) * T + t]);
+  for (int s = lane; s < nsplit; s += 32) m = fmaxf(m, part_lse[(bh * nsplit + s) * T + t]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   float acc[kPer];
 #pragma unroll
   for (int j = 0; j < kPer; ++j) acc[j] = 0.f;
   float z = 0.f;
   if (m != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      float l = part_lse[(bh * nsplit + s) * T + t];
-      if (l == -INFINITY) continue;
-      float w = expf(l - m);
-      z += w;
-      const float* src = part_o + ((bh * nsplit + s) * T + t) * D + lane * kPer;
-      if constexpr (kPer == 4) {
-        float4 v = *reinterpret_cast<const float4*>(src);
-        acc[0] += w * v.x;
-        acc[1] += w * v.y;
-        acc[2] += w * v.z;
-        acc[3] += w * v.w;
-      } else {
-        float2 v = *reinterpret_cast<const float2*>(src);
-        acc[0] += w * v.x;
-        acc[1] += w * v.y;
+    for (int s0 = 0; s0 < nsplit; s0 += 32) {
+      const int sl = s0 + lane;
+      const float l = (sl < nsplit) ? part_lse[(bh * nsplit + sl) * T + t] : -INFINITY;
+      const float wl = (l == -INFINITY) ? 0.f : expf(l - m);
+      float zs = wl;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+      z += zs;
+      const int ns = imin(32, nsplit - s0);
+#pragma unroll 4
+      for (int k = 0; k < ns; ++k) {  // independent loads: the weights are already known
+        const float w = __shfl_sync(0xffffffffu, wl, k);
+        const float* src = part_o + ((bh * nsplit + s0 + k) * T + t) * D + lane * kPer;
+        if constexpr (kPer == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(src);
+          acc[0] += w * v.x;
+          acc[1] += w * v.y;
+          acc[2] += w * v.z;
+          acc[3] += w * v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(src);
+          acc[0] += w * v.x;
+          acc[1] += w * v.y;
+        }
       }
     }
   }

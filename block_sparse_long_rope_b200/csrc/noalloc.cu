@@ -30,7 +30,7 @@
 
 #include <mutex>
 
-#include "../../include/star.h"
+#include "star.h"
 #include "star_common.cuh"
 #include "star_kernels.cuh"
 

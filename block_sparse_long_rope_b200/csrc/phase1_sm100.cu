@@ -57,6 +57,29 @@ struct AttnCfg {
   static constexpr uint32_t kTmemCols = 512;
 };
 
+// 2^x on the FMA pipe: x = n + f with n = round(x), f in [-1/2, 1/2];
+// 2^f by a degree-4 polynomial (relative error < 3e-6, fitted by
+// fit_exp2_poly.py), 2^n added to the exponent bits. x is clamped at -126
+// (the result is then < 2^-125, i.e. zero for the softmax).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;  // 1.5 * 2^23: round(x) lands in the low mantissa bits
+  const float f = x - (t - 12582912.f);
+  const int n = __float_as_int(t) - 0x4B400000;
+  float p = fmaf(9.560510516e-03f, f, 5.591703951e-02f);
+  p = fmaf(p, f, 2.402498126e-01f);
+  p = fmaf(p, f, 6.931219697e-01f);
+  p = fmaf(p, f, 9.999991655e-01f);
+  return __int_as_float(__float_as_int(p) + (n << 23));
+}
+
+// One pair of keys in kPolyEvery is exponentiated on the FMA pipe instead of
+// the MUFU unit (0 = never). The MUFU exp2 work of a KV tile equals the
+// tensor cores' MMA time at D = 128, but on B200 every tried fraction (1/8,
+// 1/4 of the pairs) cost more issue slots than it saved: 16K-context Phase 1
+// ran at 1104 / 1074 / 1012 TFLOP/s for none / 1/8 / 1/4.
+constexpr int kPolyEvery = 0;
+
 constexpr int kAttnThreads = 320;
 constexpr uint64_t kDrainNs = 100000000ull;  // 100 ms
 
@@ -247,24 +270,27 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
       w.tile(it, &key0, &lo, &hi, &causal);
       const bool full_vis =
           key0 >= lo && key0 + 128 <= hi && (!causal || key0 + 127 <= min_pos);
-      float mt = -INFINITY;
-      if (full_vis) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-          for (int j = 0; j < 32; ++j) mt = fmaxf(mt, __uint_as_float(sr[q][j]));
-      } else {
+      if (!full_vis) {
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
             const int key = key0 + 32 * q + j;
             const bool vis = key >= lo && key < hi && (!causal || key <= qpos);
-            const float v = vis ? __uint_as_float(sr[q][j]) : -INFINITY;
-            sr[q][j] = __float_as_uint(v);
-            mt = fmaxf(mt, v);
+            if (!vis) sr[q][j] = __float_as_uint(-INFINITY);
           }
       }
+      // row max: eight independent chains of 3-input max, then a tree (one
+      // chain of 128 dependent max operations would dominate the latency)
+      float mx[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) mx[j] = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          mx[j & 7] = fmax3(mx[j & 7], __uint_as_float(sr[q][2 * j]), __uint_as_float(sr[q][2 * j + 1]));
+      const float mt = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmaxf(fmax3(mx[3], mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       const float m_new = fmaxf(m_run, mt);
       if (it == 0) {
         m_run = m_new;
@@ -288,20 +314,42 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
         }
       }
       const float ref = (m_run == -INFINITY) ? 0.f : m_run * c;
-      float lsum = 0.f;
-      // P (bf16 pairs) goes back over the first 64 columns of S, 32 keys at a
-      // time; S columns 16q.. are already consumed when quarter q is written
+      // x = s * c - ref for two keys at once (fma.rn.f32x2), exp2 on the MUFU
+      // unit except every kPolyEvery-th pair (FMA pipe), row sums in four
+      // packed accumulators. P (bf16 pairs) goes back over the first 64
+      // columns of S, 32 keys at a time; S columns 16q.. are already
+      // consumed when quarter q is written.
+      const uint64_t cc = f2_pack(c, c), nref = f2_pack(-ref, -ref);
+      uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t pk[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(sr[q][2 * j]), c, -ref));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(sr[q][2 * j + 1]), c, -ref));
-          lsum += p0 + p1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[q][2 * j]), __uint_as_float(sr[q][2 * j + 1])),
+                           cc, nref), x0, x1);
+          float p0 = 0.f, p1 = 0.f;
+          bool on_fma = false;
+          if constexpr (kPolyEvery > 0) on_fma = (j % kPolyEvery) == kPolyEvery - 1;
+          if (on_fma) {
+            p0 = exp2_poly(x0);
+            p1 = exp2_poly(x1);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          ls[j & 3] = f2_add(ls[j & 3], f2_pack(p0, p1));
           pk[j] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tS + 16 * q, pk);
+      }
+      float lsum = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float a, b;
+        f2_unpack(ls[k], a, b);
+        lsum += a + b;
       }
       l_run += lsum;
       tmem_wait_st();

@@ -350,21 +350,32 @@ __global__ void __launch_bounds__(256) split_reduce_kernel(const __grid_constant
     count = p.nc_tail;
   }
   const size_t cbase = static_cast<size_t>(bh) * p.chunks_per_head + first;
+  // statistics: lanes read the chunk LSEs in parallel, shuffles reduce them
   float M = -INFINITY;
-  for (int c = 0; c < count; ++c) M = fmaxf(M, p.ws_lse[(cbase + c) * kDecRows + rho]);
+  for (int c = lane; c < count; c += 32) M = fmaxf(M, p.ws_lse[(cbase + c) * kDecRows + rho]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
   float acc[kPer];
 #pragma unroll
   for (int j = 0; j < kPer; ++j) acc[j] = 0.f;
   float z = 0.f;
   if (M != -INFINITY) {
-    for (int c = 0; c < count; ++c) {
-      const float l = p.ws_lse[(cbase + c) * kDecRows + rho];
-      if (l == -INFINITY) continue;
-      const float w = expf(l - M);
-      z += w;
-      const float* src = p.ws_o + ((cbase + c) * kDecRows + rho) * D + lane * kPer;
+    for (int c0 = 0; c0 < count; c0 += 32) {
+      const int c = c0 + lane;
+      const float l = (c < count) ? p.ws_lse[(cbase + c) * kDecRows + rho] : -INFINITY;
+      const float wl = (l == -INFINITY) ? 0.f : expf(l - M);
+      float zs = wl;
 #pragma unroll
-      for (int j = 0; j < kPer; ++j) acc[j] += w * src[j];
+      for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
+      z += zs;
+      const int nc = imin(32, count - c0);
+#pragma unroll 4
+      for (int k = 0; k < nc; ++k) {  // independent loads: the weights are already known
+        const float w = __shfl_sync(0xffffffffu, wl, k);
+        const float* src = p.ws_o + ((cbase + c0 + k) * kDecRows + rho) * D + lane * kPer;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) acc[j] += w * src[j];
+      }
     }
   }
   const float inv = (z > 0.f) ? 1.f / z : 0.f;

@@ -8,15 +8,17 @@
 // p * theta^(-2i/D).
 //
 // Precision: the angle p * theta_i, its reduction modulo 2*pi (Cody-Waite,
-// two constants), sine/cosine and the rotation are all fp64; the result is
-// rounded to bf16 once, correctly (nearest even), by rounding to fp32 with
-// round-to-odd and then to bf16 (the round-to-odd method of Boldo and
-// Melquiond, 2008: odd rounding to a format >= 2 bits wider, then nearest,
-// equals direct nearest rounding). The rotated tensors are therefore the
-// correctly rounded bf16 of the exact rotation: at p ~ 1e6 an fp32 angle
-// would err by ~0.06 rad, and even an fp32 rotation with an exact angle
-// lands one bf16 ulp off the correct value for a few elements in 1e5, enough
-// to move a peaked softmax's log-sum-exp by ~3e-2.
+// two constants) and sine/cosine are fp64. Every output is the correctly
+// rounded bf16 (nearest even) of the exact rotation. The rotation first runs
+// in fp32 with a bound E on its error; when y - E and y + E round to the same
+// bf16 value that value is the correct rounding (Ziv's rounding test), and
+// otherwise (about one element in 10^4) the element is recomputed in fp64 and
+// rounded once through fp32 round-to-odd (Boldo and Melquiond, 2008: odd
+// rounding to a format >= 2 bits wider, then nearest, equals direct nearest
+// rounding). At p ~ 1e6 an fp32 angle would err by ~0.06 rad, and even an
+// fp32 rotation with an exact angle lands one bf16 ulp off the correct value
+// for a few elements in 1e5, enough to move a peaked softmax's log-sum-exp by
+// ~3e-2; correct rounding makes the cache reproducible bit for bit.
 // theta_i = theta^(-2i/D) comes from the host in fp64.
 //
 // One launch handles up to three jobs (Q, K, V of one call): blockIdx.z
@@ -56,6 +58,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
 
   __shared__ double s_cos[kTokPerCta][64];
   __shared__ double s_sin[kTokPerCta][64];
+  __shared__ float f_cos[kTokPerCta][64];
+  __shared__ float f_sin[kTokPerCta][64];
   if (job.rotate) {
     for (int e = threadIdx.x; e < ntok * half; e += blockDim.x) {
       int t = e / half, i = e % half;
@@ -69,6 +73,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
       sincos(r, &sn, &cs);
       s_cos[t][i] = cs;
       s_sin[t][i] = sn;
+      f_cos[t][i] = static_cast<float>(cs);
+      f_sin[t][i] = static_cast<float>(sn);
     }
     __syncthreads();
   }
@@ -89,13 +95,34 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
       uint32_t ol[4], oh[4];
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
-        int i0 = 8 * c + 2 * w;
-        double a0 = bf16_lo(pl[w]), a1 = bf16_hi(pl[w]);
-        double b0 = bf16_lo(ph[w]), b1 = bf16_hi(ph[w]);
-        double c0 = s_cos[t][i0], c1 = s_cos[t][i0 + 1];
-        double s0 = s_sin[t][i0], s1 = s_sin[t][i0 + 1];
-        ol[w] = pack_bf16x2(f32_round_odd(a0 * c0 - b0 * s0), f32_round_odd(a1 * c1 - b1 * s1));
-        oh[w] = pack_bf16x2(f32_round_odd(b0 * c0 + a0 * s0), f32_round_odd(b1 * c1 + a1 * s1));
+        const int i0 = 8 * c + 2 * w;
+        const float a0 = bf16_lo(pl[w]), a1 = bf16_hi(pl[w]);
+        const float b0 = bf16_lo(ph[w]), b1 = bf16_hi(ph[w]);
+        const float c0 = f_cos[t][i0], c1 = f_cos[t][i0 + 1];
+        const float s0 = f_sin[t][i0], s1 = f_sin[t][i0 + 1];
+        // |fp32 result - exact| <= 2^-22 (|a| + |b|): one rounding each for
+        // cos/sin (2^-25 relative), the product and the fused multiply-add
+        const float e0 = 2.3841858e-07f * (fabsf(a0) + fabsf(b0));
+        const float e1 = 2.3841858e-07f * (fabsf(a1) + fabsf(b1));
+        float y[4] = {fmaf(a0, c0, -(b0 * s0)), fmaf(a1, c1, -(b1 * s1)),
+                      fmaf(b0, c0, a0 * s0), fmaf(b1, c1, a1 * s1)};
+        const float err[4] = {e0, e1, e0, e1};
+        uint32_t out[4];
+#pragma unroll
+        for (int m = 0; m < 4; ++m) {
+          const uint32_t lohi = pack_bf16x2(y[m] - err[m], y[m] + err[m]);
+          if ((lohi & 0xFFFFu) == (lohi >> 16)) {
+            out[m] = lohi & 0xFFFFu;
+          } else {  // within E of a rounding boundary: decide in fp64
+            const int ii = i0 + (m & 1);
+            const double ad = (m & 1) ? a1 : a0, bd = (m & 1) ? b1 : b0;
+            const double cd = s_cos[t][ii], sd = s_sin[t][ii];
+            const double yd = (m < 2) ? ad * cd - bd * sd : bd * cd + ad * sd;
+            out[m] = pack_bf16x2(f32_round_odd(yd), 0.f) & 0xFFFFu;
+          }
+        }
+        ol[w] = out[0] | (out[1] << 16);
+        oh[w] = out[2] | (out[3] << 16);
       }
       lo = make_uint4(ol[0], ol[1], ol[2], ol[3]);
       hi = make_uint4(oh[0], oh[1], oh[2], oh[3]);

@@ -74,9 +74,8 @@ const char* star_version(void);
  * x, y: bf16, D contiguous; x_stride / y_stride give the element strides of
  * the (B, S, H) dimensions (each a multiple of 8). x and y may be the same
  * buffer (in place) but must not otherwise overlap. pos: device int32[S] or
- * NULL. The angle p * theta_i is formed and reduced modulo 2*pi in fp64;
- * sine/cosine and the rotation run in fp32; y is rounded to bf16 (nearest
- * even).
+ * NULL. Angles, their reduction modulo 2*pi and sine/cosine are fp64; y is
+ * the correctly rounded bf16 (nearest even) of the exact rotation.
  */
 star_status star_rope(const void* x, const int64_t x_stride[3], void* y,
                       const int64_t y_stride[3], const int32_t* pos, int64_t pos0, int B,
