@@ -155,7 +155,35 @@ int decode_chunks_per_head(int L, int b, int n, int tail_plus_T, int chunk, int*
   return (n - 1) * *nc_full + *nc_last + *nc_tail;
 }
 constexpr int kMinChunk = 256;
-constexpr int kMaxChunk = 4096;
+constexpr int kMaxChunk = 65536;
+
+int next_pow2(int x) {
+  int p = 1;
+  while (p < x) p <<= 1;
+  return p;
+}
+
+// Keys per decode CTA: long enough that a split has at most
+// kMaxChunksPerSplit chunks (the last CTA of a split reduces them), then as
+// long as the grid still gives every SM two CTAs.
+int decode_chunk(int B, int Hkv, int L, int b, int n, int tail_plus_T, int sms) {
+  const int max_split = star::imax(imin(b, L), tail_plus_T);
+  int chunk = star::imax(kMinChunk, next_pow2(ceil_div(max_split, star::kMaxChunksPerSplit)));
+  const int cap = imin(kMaxChunk, next_pow2(max_split));
+  int nf, nl, nt;
+  while (chunk * 2 <= cap &&
+         (long long)B * Hkv * decode_chunks_per_head(L, b, n, tail_plus_T, chunk * 2, &nf, &nl, &nt) >=
+             2ll * sms)
+    chunk *= 2;
+  return chunk;
+}
+
+// Bytes of the zeroed header of a decode workspace: the status word, then
+// one finished-chunk counter per (batch, KV head, split).
+size_t decode_header_bytes(int B, int Hkv, int Lcap, int block_len) {
+  const long long nsplit_cap = ceil_div(Lcap, block_len) + 1;
+  return star::kStatusBytes + align_up((size_t)B * Hkv * nsplit_cap * sizeof(int));
+}
 
 bool use_decode_path(int T, int Hq, int Hkv) {
   const int g = Hq / Hkv;
@@ -309,9 +337,10 @@ star_status star_phase1_encode(const void* q, const void* k, const void* v, void
 size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lcap, int block_len) {
   if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || D < 1 || Lcap < 1 || block_len < 1 || Hq % Hkv)
     return star::kStatusBytes;
-  size_t bytes = star::kStatusBytes + align_up((size_t)B * T * Hq * D * 2);
-  if (use_decode_path(T, Hq, Hkv)) bytes += decode_scratch_bytes(B, Hkv, D, Lcap, block_len);
-  return bytes;
+  if (use_decode_path(T, Hq, Hkv))
+    return decode_header_bytes(B, Hkv, Lcap, block_len) + align_up((size_t)B * T * Hq * D * 2) +
+           decode_scratch_bytes(B, Hkv, D, Lcap, block_len);
+  return star::kStatusBytes + align_up((size_t)B * T * Hq * D * 2);
 }
 
 star_status star_phase2_partial(const void* q, const void* k, const void* v, int T, void* k_cache,
@@ -343,9 +372,12 @@ star_status star_phase2_partial(const void* q, const void* k, const void* v, int
 
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  __nv_bfloat16* qrot = reinterpret_cast<__nv_bfloat16*>(ws + star::kStatusBytes);
+  const bool decode = use_decode_path(T, Hq, Hkv);
+  // zeroed header (status word; split counters on the decode path), then the rotated q
+  const size_t header = decode ? decode_header_bytes(B, Hkv, Lcap, block_len) : star::kStatusBytes;
+  __nv_bfloat16* qrot = reinterpret_cast<__nv_bfloat16*>(ws + header);
   const size_t qrot_bytes = align_up((size_t)B * T * Hq * D * 2);
-  cudaError_t e = cudaMemsetAsync(ws, 0, star::kStatusBytes, st);
+  cudaError_t e = cudaMemsetAsync(ws, 0, header, st);
   if (e != cudaSuccess) return cuda_fail(e, "status reset");
 
   // RoPE of the new tokens at positions L + tail_len + t; K/V appended to the
@@ -378,7 +410,7 @@ star_status star_phase2_partial(const void* q, const void* k, const void* v, int
   const int g = Hq / Hkv;
   if (nsplit_out) *nsplit_out = nsplit;
 
-  if (use_decode_path(T, Hq, Hkv)) {
+  if (decode) {
     star::DecodeParams dp;
     memset(&dp, 0, sizeof dp);
     if ((s = map_cache(&dp.tmK, k_cache, B * Hkv, Lcap, valid, D, star::kDecTile)) != STAR_OK) return s;
@@ -394,20 +426,14 @@ star_status star_phase2_partial(const void* q, const void* k, const void* v, int
     dp.b = block_len;
     dp.n = n;
     dp.tail_len = tail_len;
-    // smallest chunk that still gives every SM several CTAs
-    int chunk = kMinChunk;
-    int nf, nl, nt;
-    while (chunk < kMaxChunk &&
-           (long long)B * Hkv * decode_chunks_per_head(L, block_len, n, tail_len + T, chunk * 2, &nf, &nl, &nt) >=
-               8ll * sms)
-      chunk *= 2;
+    const int chunk = decode_chunk(B, Hkv, L, block_len, n, tail_len + T, sms);
     dp.chunk = chunk;
     dp.chunks_per_head = decode_chunks_per_head(L, block_len, n, tail_len + T, chunk, &dp.nc_full,
                                                 &dp.nc_last, &dp.nc_tail);
     const size_t rows = (size_t)B * Hkv * dp.chunks_per_head * star::kDecRows;
-    dp.ws_o = reinterpret_cast<float*>(ws + star::kStatusBytes + qrot_bytes);
-    dp.ws_lse = reinterpret_cast<float*>(ws + star::kStatusBytes + qrot_bytes +
-                                         align_up(rows * D * sizeof(float)));
+    dp.ws_o = reinterpret_cast<float*>(ws + header + qrot_bytes);
+    dp.ws_lse = reinterpret_cast<float*>(ws + header + qrot_bytes + align_up(rows * D * sizeof(float)));
+    dp.counters = reinterpret_cast<int*>(ws + star::kStatusBytes);
     dp.part_o = part_o;
     dp.part_lse = part_lse;
     dp.status = reinterpret_cast<int*>(ws);

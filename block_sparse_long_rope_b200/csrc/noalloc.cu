@@ -15,8 +15,9 @@
 //    call made with that device current (cudaGetSymbolAddress). Make that
 //    first call before any stream capture.
 //  * Every call on a device shares the one array and it keeps the previous
-//    call's contents. The status word at its start is cleared by every call;
-//    everything else is fully rewritten before it is read. Calls whose work
+//    call's contents. The status word and the per-split chunk counters at
+//    its start are cleared by every call; everything else is fully
+//    rewritten before it is read. Calls whose work
 //    overlaps on the GPU (different streams, or host threads without
 //    ordering) race on the array: serialise them.
 //  * Sizes that cannot fit are rejected with STAR_ERR_INVALID_ARG before
@@ -163,9 +164,11 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
 
   // scratch layout and chunk size: the smallest chunk (>= 256 keys) that both
   // fits the array and leaves several CTAs per SM
-  const size_t qrot_bytes = align256((size_t)B * T * Hq * D * 2);
-  const size_t head_bytes = star::kStatusBytes + qrot_bytes;
   const int n = star::ceil_div(L, block_len);
+  const size_t qrot_bytes = align256((size_t)B * T * Hq * D * 2);
+  // zeroed header: status word, then one finished-chunk counter per split
+  const size_t zero_bytes = star::kStatusBytes + align256((size_t)B * Hkv * (n + 1) * sizeof(int));
+  const size_t head_bytes = zero_bytes + qrot_bytes;
   void* base = nullptr;
   int sms = 148;
   star_status st = scratch_address(&base, &sms);
@@ -177,24 +180,29 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
     return head_bytes + align256(rows * D * sizeof(float)) + align256(rows * sizeof(float)) <=
            kStaticScratchBytes;
   };
+  // at most kMaxChunksPerSplit chunks per split (the last CTA of a split
+  // reduces them), large enough to fit the array, then as long as the grid
+  // still gives every SM two CTAs
+  const int max_split = star::imax(star::imin(block_len, L), tail_len + T);
   int chunk = kMinChunk;
-  while (chunk < kMaxChunk && !fits(chunk)) chunk *= 2;
-  if (!fits(chunk))
+  while (chunk < kMaxChunk && (star::ceil_div(max_split, chunk) > star::kMaxChunksPerSplit || !fits(chunk)))
+    chunk *= 2;
+  if (!fits(chunk) || star::ceil_div(max_split, chunk) > star::kMaxChunksPerSplit)
     return fail_static(STAR_ERR_INVALID_ARG,
                        "problem needs more than the %zu-byte static scratch (B=%d Hkv=%d L=%d)",
                        kStaticScratchBytes, B, Hkv, L);
-  while (chunk < kMaxChunk) {
+  while (chunk * 2 <= kMaxChunk && chunk < max_split) {
     int a, b, c;
     long long ctas = (long long)B * Hkv * chunks_per_head(L, block_len, n, tail_len + T, chunk * 2, &a, &b, &c);
-    if (ctas < 8ll * sms) break;
+    if (ctas < 2ll * sms) break;
     chunk *= 2;
   }
 
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   unsigned char* ws = static_cast<unsigned char*>(base);
-  cudaError_t e = cudaMemsetAsync(ws, 0, star::kStatusBytes, stream);
+  cudaError_t e = cudaMemsetAsync(ws, 0, zero_bytes, stream);
   if (e != cudaSuccess) return fail_static(STAR_ERR_CUDA, "status reset: %s", cudaGetErrorString(e));
-  __nv_bfloat16* qrot = reinterpret_cast<__nv_bfloat16*>(ws + star::kStatusBytes);
+  __nv_bfloat16* qrot = reinterpret_cast<__nv_bfloat16*>(ws + zero_bytes);
 
   // RoPE of the new tokens; K/V appended to the cache rows L + tail_len + t
   const int row0 = L + tail_len;
@@ -244,6 +252,7 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
   dp.part_o = part_o;
   dp.part_lse = part_lse;
   dp.status = reinterpret_cast<int*>(ws);
+  dp.counters = reinterpret_cast<int*>(ws + star::kStatusBytes);
   dp.scale_ln = (float)(1.0 / sqrt((double)D));
   dp.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   e = star::launch_decode(dp, D, stream);

@@ -10,8 +10,8 @@
 //    so each K/V byte is read once for all g heads of its group.
 //  * A split is cut into chunks of `chunk` keys, one CTA each, so that the
 //    grid covers all 148 SMs even when (batch x KV heads x blocks) is small.
-//    CTAs reduce their chunk in-kernel; a second small kernel combines the
-//    chunks of a split in fixed order (deterministic).
+//    CTAs reduce their chunk in-kernel; the last CTA to finish a chunk of a
+//    split combines that split's chunks in fixed order (deterministic).
 //  * A producer warp streams 64-key K/V tiles with TMA (128-byte swizzle)
 //    into a 3-stage shared-memory ring; four consumer warps each own 16 keys
 //    of a tile.
@@ -95,6 +95,63 @@ __device__ __forceinline__ ChunkRange chunk_range(const DecodeParams& p, int c) 
 }
 
 }  // namespace
+
+// Reduce the chunk partials of one split (fixed order) into part_o /
+// part_lse. Run by the last CTA that finished a chunk of the split; `sw` is
+// free shared memory (>= kDecRows * (kMaxChunksPerSplit + 2) floats).
+template <int D>
+__device__ void reduce_split(const DecodeParams& p, int bh, int split, float* sw) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int nwarps = blockDim.x / 32;
+  const int nsplit = p.n + 1;
+  int first, count;
+  if (split < p.n - 1) {
+    first = split * p.nc_full;
+    count = p.nc_full;
+  } else if (split == p.n - 1) {
+    first = (p.n - 1) * p.nc_full;
+    count = p.nc_last;
+  } else {
+    first = (p.n - 1) * p.nc_full + p.nc_last;
+    count = p.nc_tail;
+  }
+  const size_t cbase = static_cast<size_t>(bh) * p.chunks_per_head + first;
+  float* wgt = sw;                          // [R][count] weights exp(lse_c - M)
+  float* rowz = sw + kDecRows * kMaxChunksPerSplit;  // [R] sum of weights
+  float* rowm = rowz + kDecRows;            // [R] max statistic
+  for (int rho = warp; rho < p.R; rho += nwarps) {
+    float M = -INFINITY;
+    for (int c = lane; c < count; c += 32) M = fmaxf(M, p.ws_lse[(cbase + c) * kDecRows + rho]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float z = 0.f;
+    for (int c = lane; c < count; c += 32) {
+      const float l = p.ws_lse[(cbase + c) * kDecRows + rho];
+      const float wv = (M == -INFINITY || l == -INFINITY) ? 0.f : expf(l - M);
+      wgt[rho * kMaxChunksPerSplit + c] = wv;
+      z += wv;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane == 0) {
+      rowz[rho] = z;
+      rowm[rho] = M;
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < p.R * D; idx += blockDim.x) {
+    const int rho = idx / D, d = idx % D;
+    float acc = 0.f;
+    for (int c = 0; c < count; ++c)  // independent loads: the weights are known
+      acc += wgt[rho * kMaxChunksPerSplit + c] * p.ws_o[((cbase + c) * kDecRows + rho) * D + d];
+    const float z = rowz[rho];
+    const int t = rho / p.g, h = (bh % p.Hkv) * p.g + rho % p.g;
+    const int b = bh / p.Hkv;
+    const size_t row = ((static_cast<size_t>(b) * p.Hq + h) * nsplit + split) * p.T + t;
+    p.part_o[row * D + d] = (z > 0.f) ? acc / z : 0.f;
+    if (d == 0) p.part_lse[row] = (z > 0.f) ? rowm[rho] + logf(z) : -INFINITY;
+  }
+}
 
 template <int D>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_constant__ DecodeParams p) {
@@ -323,68 +380,20 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     p.ws_o[(base * kDecRows + rho) * D + d] = out;
     if (d == 0) p.ws_lse[base * kDecRows + rho] = lse;
   }
-}
-
-// Combine the chunks of each split (fixed order) into part_o / part_lse.
-template <int D>
-__global__ void __launch_bounds__(256) split_reduce_kernel(const __grid_constant__ DecodeParams p) {
-  constexpr int kPer = D / 32;
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
-  const int lane = threadIdx.x % 32;
-  const int nsplit = p.n + 1;
-  const int total = p.B * p.Hkv * nsplit * p.R;
-  if (warp >= total) return;
-  const int rho = warp % p.R;
-  const int split = (warp / p.R) % nsplit;
-  const int bh = warp / (p.R * nsplit);
-  const int b = bh / p.Hkv, kvh = bh % p.Hkv;
-  int first, count;
-  if (split < p.n - 1) {
-    first = split * p.nc_full;
-    count = p.nc_full;
-  } else if (split == p.n - 1) {
-    first = (p.n - 1) * p.nc_full;
-    count = p.nc_last;
-  } else {
-    first = (p.n - 1) * p.nc_full + p.nc_last;
-    count = p.nc_tail;
+  // The last CTA to finish a chunk of this split reduces the split: every
+  // CTA publishes its partial (fence) before counting itself in.
+  __shared__ int is_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const int prev = atomicAdd(&p.counters[bh * (p.n + 1) + cr.split], 1);
+    const int in_split = cr.split < p.n - 1 ? p.nc_full : (cr.split == p.n - 1 ? p.nc_last : p.nc_tail);
+    is_last = (prev == in_split - 1);
   }
-  const size_t cbase = static_cast<size_t>(bh) * p.chunks_per_head + first;
-  // statistics: lanes read the chunk LSEs in parallel, shuffles reduce them
-  float M = -INFINITY;
-  for (int c = lane; c < count; c += 32) M = fmaxf(M, p.ws_lse[(cbase + c) * kDecRows + rho]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-  float acc[kPer];
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) acc[j] = 0.f;
-  float z = 0.f;
-  if (M != -INFINITY) {
-    for (int c0 = 0; c0 < count; c0 += 32) {
-      const int c = c0 + lane;
-      const float l = (c < count) ? p.ws_lse[(cbase + c) * kDecRows + rho] : -INFINITY;
-      const float wl = (l == -INFINITY) ? 0.f : expf(l - M);
-      float zs = wl;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
-      z += zs;
-      const int nc = imin(32, count - c0);
-#pragma unroll 4
-      for (int k = 0; k < nc; ++k) {  // independent loads: the weights are already known
-        const float w = __shfl_sync(0xffffffffu, wl, k);
-        const float* src = p.ws_o + ((cbase + c0 + k) * kDecRows + rho) * D + lane * kPer;
-#pragma unroll
-        for (int j = 0; j < kPer; ++j) acc[j] += w * src[j];
-      }
-    }
-  }
-  const float inv = (z > 0.f) ? 1.f / z : 0.f;
-  const int t = rho / p.g, h = kvh * p.g + rho % p.g;
-  const size_t row = ((static_cast<size_t>(b) * p.Hq + h) * nsplit + split) * p.T + t;
-  float* dst = p.part_o + row * D + lane * kPer;
-#pragma unroll
-  for (int j = 0; j < kPer; ++j) dst[j] = acc[j] * inv;
-  if (lane == 0) p.part_lse[row] = (z > 0.f) ? M + logf(z) : -INFINITY;
+  __syncthreads();
+  if (!is_last) return;
+  __threadfence();
+  reduce_split<D>(p, bh, cr.split, reinterpret_cast<float*>(sm));
 }
 
 size_t decode_smem_bytes(int D) {
@@ -395,37 +404,21 @@ size_t decode_smem_bytes(int D) {
 cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t stream) {
   const int units = p.B * p.Hkv * p.chunks_per_head;
   const size_t smem = decode_smem_bytes(D);
-  const int warps = p.B * p.Hkv * (p.n + 1) * p.R;
-  const int rblocks = ceil_div(warps * 32, 256);
   int dev = 0;
   cudaGetDevice(&dev);
-  if (D == 128) {
-    static bool attr[64] = {};
-    if (dev >= 64 || !attr[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(decode_kernel<128>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      if (dev < 64) attr[dev] = true;
-    }
-    decode_kernel<128><<<units, kDecThreads, smem, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
+  static bool attr128[64] = {}, attr64[64] = {};
+  bool* attr = (D == 128) ? attr128 : attr64;
+  if (dev >= 64 || !attr[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(D == 128 ? decode_kernel<128> : decode_kernel<64>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    split_reduce_kernel<128><<<rblocks, 256, 0, stream>>>(p);
-  } else {
-    static bool attr[64] = {};
-    if (dev >= 64 || !attr[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(decode_kernel<64>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      if (dev < 64) attr[dev] = true;
-    }
-    decode_kernel<64><<<units, kDecThreads, smem, stream>>>(p);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return e;
-    split_reduce_kernel<64><<<rblocks, 256, 0, stream>>>(p);
+    if (dev < 64) attr[dev] = true;
   }
+  if (D == 128)
+    decode_kernel<128><<<units, kDecThreads, smem, stream>>>(p);
+  else
+    decode_kernel<64><<<units, kDecThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 
