@@ -29,6 +29,7 @@ EXPORTS = (
     "star_phase2_workspace_bytes",
     "star_phase2_partial",
     "star_phase2_decode_static",
+    "star_phase2_attend",
     "star_lse_merge",
     "star_device_status",
     "star_debug_index",
@@ -84,6 +85,9 @@ def load(path: str = LIB_PATH):
         lib.star_phase2_decode_static.restype = _I
         lib.star_phase2_decode_static.argtypes = [_P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P,
                                                   _IP, _I, _I, _I, _I, _D, _P]
+        lib.star_phase2_attend.restype = _I
+        lib.star_phase2_attend.argtypes = [_P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P,
+                                           _IP, _I, _I, _I, _I, _D, _P, _SZ, _P]
         lib.star_lse_merge.restype = _I
         lib.star_lse_merge.argtypes = [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P]
         lib.star_device_status.restype = _I

@@ -9,6 +9,7 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <algorithm>
 #include <mutex>
 #include <string>
 
@@ -154,35 +155,38 @@ int decode_chunks_per_head(int L, int b, int n, int tail_plus_T, int chunk, int*
   *nc_tail = ceil_div(tail_plus_T, chunk);
   return (n - 1) * *nc_full + *nc_last + *nc_tail;
 }
-constexpr int kMinChunk = 256;
-constexpr int kMaxChunk = 65536;
 
-int next_pow2(int x) {
-  int p = 1;
-  while (p < x) p <<= 1;
-  return p;
-}
-
-// Keys per decode CTA: long enough that a split has at most
-// kMaxChunksPerSplit chunks (the last CTA of a split reduces them), then as
-// long as the grid still gives every SM two CTAs.
+// Keys per decode work unit (a multiple of the 64-key tile). The grid is two
+// persistent CTAs per SM; units are sized so that all of them fit in that
+// one wave with equal work (the total tiles of all splits divided over the
+// CTAs left after one extra unit per split for the ragged ends), and so that
+// a split has at most kMaxChunksPerSplit units. When there are more splits
+// than CTAs every split is one unit and CTAs loop over several.
 int decode_chunk(int B, int Hkv, int L, int b, int n, int tail_plus_T, int sms) {
-  const int max_split = star::imax(imin(b, L), tail_plus_T);
-  int chunk = star::imax(kMinChunk, next_pow2(ceil_div(max_split, star::kMaxChunksPerSplit)));
-  const int cap = imin(kMaxChunk, next_pow2(max_split));
-  int nf, nl, nt;
-  while (chunk * 2 <= cap &&
-         (long long)B * Hkv * decode_chunks_per_head(L, b, n, tail_plus_T, chunk * 2, &nf, &nl, &nt) >=
-             2ll * sms)
-    chunk *= 2;
-  return chunk;
+  const int tile = star::kDecTile;
+  const long long tiles_head = (long long)(n - 1) * ceil_div(imin(b, L), tile) +
+                               ceil_div(L - (n - 1) * b, tile) + ceil_div(tail_plus_T, tile);
+  const long long total_tiles = tiles_head * B * Hkv;
+  const long long splits = (long long)B * Hkv * (n + 1);
+  const long long ctas = 2ll * sms;
+  const long long room = ctas - splits;
+  const int max_split_tiles = ceil_div(star::imax(imin(b, L), tail_plus_T), tile);
+  long long chunk_tiles = room > 0 ? (total_tiles + room - 1) / room : max_split_tiles;
+  chunk_tiles = std::max<long long>(chunk_tiles, ceil_div(max_split_tiles, star::kMaxChunksPerSplit));
+  chunk_tiles = std::max<long long>(1, std::min<long long>(chunk_tiles, max_split_tiles));
+  return static_cast<int>(chunk_tiles) * tile;
 }
 
-// Bytes of the zeroed header of a decode workspace: the status word, then
-// one finished-chunk counter per (batch, KV head, split).
-size_t decode_header_bytes(int B, int Hkv, int Lcap, int block_len) {
+// Bytes of the zeroed header of a decode workspace: the status word, one
+// finished-chunk counter per (batch, KV head, split), then one finished-split
+// counter per (batch, KV head).
+size_t decode_split_counter_bytes(int B, int Hkv, int Lcap, int block_len) {
   const long long nsplit_cap = ceil_div(Lcap, block_len) + 1;
-  return star::kStatusBytes + align_up((size_t)B * Hkv * nsplit_cap * sizeof(int));
+  return align_up((size_t)B * Hkv * nsplit_cap * sizeof(int));
+}
+size_t decode_header_bytes(int B, int Hkv, int Lcap, int block_len) {
+  return star::kStatusBytes + decode_split_counter_bytes(B, Hkv, Lcap, block_len) +
+         align_up((size_t)B * Hkv * sizeof(int));
 }
 
 bool use_decode_path(int T, int Hq, int Hkv) {
@@ -191,10 +195,11 @@ bool use_decode_path(int T, int Hq, int Hkv) {
 }
 
 size_t decode_scratch_bytes(int B, int Hkv, int D, int Lcap, int block_len) {
-  // worst case over L + tail <= Lcap at the smallest chunk
-  const long long nsplit_max = ceil_div(Lcap, block_len) + 1;
-  const long long cph = ceil_div(Lcap, kMinChunk) + nsplit_max;
-  const long long rows = (long long)B * Hkv * cph * star::kDecRows;
+  // decode_chunk makes at most max(2 * SMs, splits) + splits units for any
+  // L + tail <= Lcap (one extra per split for its ragged end); SMs <= 256
+  const long long splits = (long long)B * Hkv * (ceil_div(Lcap, block_len) + 1);
+  const long long units = std::max<long long>(512, splits) + splits;
+  const long long rows = units * star::kDecRows;
   return align_up((size_t)rows * D * sizeof(float)) + align_up((size_t)rows * sizeof(float));
 }
 
@@ -343,11 +348,16 @@ size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lca
   return star::kStatusBytes + align_up((size_t)B * T * Hq * D * 2);
 }
 
-star_status star_phase2_partial(const void* q, const void* k, const void* v, int T, void* k_cache,
-                                void* v_cache, int Lcap, int L, int block_len, int tail_len,
-                                float* part_o, float* part_lse, int* nsplit_out, int B, int Hq,
-                                int Hkv, int D, double theta, void* workspace,
-                                size_t workspace_bytes, void* cuda_stream) {
+}  // extern "C"
+
+namespace {
+
+// Body of star_phase2_partial / star_phase2_attend; o_merged == NULL skips the merge.
+star_status phase2_run(const void* q, const void* k, const void* v, int T, void* k_cache,
+                       void* v_cache, int Lcap, int L, int block_len, int tail_len, float* part_o,
+                       float* part_lse, void* o_merged, float* lse_merged, int* nsplit_out, int B,
+                       int Hq, int Hkv, int D, double theta, void* workspace,
+                       size_t workspace_bytes, void* cuda_stream) {
   star_status s;
   if ((s = check_heads(B, Hq, Hkv, D)) != STAR_OK) return s;
   if (T < 1) return fail(STAR_ERR_INVALID_ARG, "T must be >= 1");
@@ -364,6 +374,10 @@ star_status star_phase2_partial(const void* q, const void* k, const void* v, int
     return s;
   if (!part_lse || (reinterpret_cast<uintptr_t>(part_lse) & 3u))
     return fail(STAR_ERR_INVALID_ARG, "part_lse is NULL or not 4-byte aligned");
+  if (o_merged && !aligned16(o_merged))
+    return fail(STAR_ERR_INVALID_ARG, "o is not 16-byte aligned");
+  if (lse_merged && (reinterpret_cast<uintptr_t>(lse_merged) & 3u))
+    return fail(STAR_ERR_INVALID_ARG, "lse is not 4-byte aligned");
   const size_t need = star_phase2_workspace_bytes(B, T, Hq, Hkv, D, Lcap, block_len);
   if (workspace_bytes < need)
     return fail(STAR_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
@@ -434,6 +448,10 @@ star_status star_phase2_partial(const void* q, const void* k, const void* v, int
     dp.ws_o = reinterpret_cast<float*>(ws + header + qrot_bytes);
     dp.ws_lse = reinterpret_cast<float*>(ws + header + qrot_bytes + align_up(rows * D * sizeof(float)));
     dp.counters = reinterpret_cast<int*>(ws + star::kStatusBytes);
+    dp.head_counters = reinterpret_cast<int*>(ws + star::kStatusBytes +
+                                              decode_split_counter_bytes(B, Hkv, Lcap, block_len));
+    dp.o_merged = static_cast<__nv_bfloat16*>(o_merged);
+    dp.lse_merged = lse_merged;
     dp.part_o = part_o;
     dp.part_lse = part_lse;
     dp.status = reinterpret_cast<int*>(ws);
@@ -470,7 +488,37 @@ star_status star_phase2_partial(const void* q, const void* k, const void* v, int
   ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   e = star::launch_attn(ap, D, st);
   if (e != cudaSuccess) return cuda_fail(e, "phase-2 chunk attention launch");
+  if (o_merged) {
+    e = star::launch_lse_merge(part_o, part_lse, nsplit, static_cast<__nv_bfloat16*>(o_merged),
+                               lse_merged, B, T, Hq, D, st);
+    if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
+  }
   return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+star_status star_phase2_partial(const void* q, const void* k, const void* v, int T, void* k_cache,
+                                void* v_cache, int Lcap, int L, int block_len, int tail_len,
+                                float* part_o, float* part_lse, int* nsplit_out, int B, int Hq,
+                                int Hkv, int D, double theta, void* workspace,
+                                size_t workspace_bytes, void* cuda_stream) {
+  return phase2_run(q, k, v, T, k_cache, v_cache, Lcap, L, block_len, tail_len, part_o, part_lse,
+                    nullptr, nullptr, nsplit_out, B, Hq, Hkv, D, theta, workspace,
+                    workspace_bytes, cuda_stream);
+}
+
+star_status star_phase2_attend(const void* q, const void* k, const void* v, int T, void* k_cache,
+                               void* v_cache, int Lcap, int L, int block_len, int tail_len,
+                               float* part_o, float* part_lse, void* o, float* lse,
+                               int* nsplit_out, int B, int Hq, int Hkv, int D, double theta,
+                               void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  if (!o) return fail(STAR_ERR_INVALID_ARG, "o is NULL");
+  return phase2_run(q, k, v, T, k_cache, v_cache, Lcap, L, block_len, tail_len, part_o, part_lse,
+                    o, lse, nsplit_out, B, Hq, Hkv, D, theta, workspace, workspace_bytes,
+                    cuda_stream);
 }
 
 star_status star_lse_merge(const float* part_o, const float* part_lse, int nsplit, void* o,

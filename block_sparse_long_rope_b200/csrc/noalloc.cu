@@ -167,7 +167,8 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
   const int n = star::ceil_div(L, block_len);
   const size_t qrot_bytes = align256((size_t)B * T * Hq * D * 2);
   // zeroed header: status word, then one finished-chunk counter per split
-  const size_t zero_bytes = star::kStatusBytes + align256((size_t)B * Hkv * (n + 1) * sizeof(int));
+  const size_t zero_bytes = star::kStatusBytes + align256((size_t)B * Hkv * (n + 1) * sizeof(int)) +
+                            align256((size_t)B * Hkv * sizeof(int));
   const size_t head_bytes = zero_bytes + qrot_bytes;
   void* base = nullptr;
   int sms = 148;
@@ -180,9 +181,9 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
     return head_bytes + align256(rows * D * sizeof(float)) + align256(rows * sizeof(float)) <=
            kStaticScratchBytes;
   };
-  // at most kMaxChunksPerSplit chunks per split (the last CTA of a split
-  // reduces them), large enough to fit the array, then as long as the grid
-  // still gives every SM two CTAs
+  // at most kMaxChunksPerSplit chunks per split (the CTA completing a split
+  // reduces them), large enough to fit the array, then doubled while every
+  // persistent CTA still gets several units
   const int max_split = star::imax(star::imin(block_len, L), tail_len + T);
   int chunk = kMinChunk;
   while (chunk < kMaxChunk && (star::ceil_div(max_split, chunk) > star::kMaxChunksPerSplit || !fits(chunk)))
@@ -193,8 +194,8 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
                        kStaticScratchBytes, B, Hkv, L);
   while (chunk * 2 <= kMaxChunk && chunk < max_split) {
     int a, b, c;
-    long long ctas = (long long)B * Hkv * chunks_per_head(L, block_len, n, tail_len + T, chunk * 2, &a, &b, &c);
-    if (ctas < 2ll * sms) break;
+    long long units = (long long)B * Hkv * chunks_per_head(L, block_len, n, tail_len + T, chunk * 2, &a, &b, &c);
+    if (units < 16ll * sms) break;  // keep >= 8 units per persistent CTA
     chunk *= 2;
   }
 

@@ -8,10 +8,12 @@
 // HBM-bound: every step streams the whole K/V cache once. Design:
 //  * The T*g (token, query-head) rows of one GQA group form one 16-row tile,
 //    so each K/V byte is read once for all g heads of its group.
-//  * A split is cut into chunks of `chunk` keys, one CTA each, so that the
-//    grid covers all 148 SMs even when (batch x KV heads x blocks) is small.
-//    CTAs reduce their chunk in-kernel; the last CTA to finish a chunk of a
-//    split combines that split's chunks in fixed order (deterministic).
+//  * A split is cut into chunks of `chunk` keys; the (head, chunk) units are
+//    spread over a persistent grid of two CTAs per SM, each streaming a
+//    contiguous run of units without a pause between them. A CTA reduces
+//    each chunk in-kernel; the CTA completing a split's last chunk combines
+//    that split's chunks in fixed order (deterministic), and the CTA
+//    completing a head's last split merges the splits when asked to.
 //  * A producer warp streams 64-key K/V tiles with TMA (128-byte swizzle)
 //    into a 3-stage shared-memory ring; four consumer warps each own 16 keys
 //    of a tile.
@@ -96,30 +98,55 @@ __device__ __forceinline__ ChunkRange chunk_range(const DecodeParams& p, int c) 
 
 }  // namespace
 
+constexpr int kConsumers = 128;  // threads of the four consumer warps
+
+// Barrier among the four consumer warps only (the producer warp runs ahead).
+__device__ __forceinline__ void consumer_sync() {
+  asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+// Consumer barrier that also returns whether any consumer thread passed a
+// non-zero flag: every consumer warp takes the same branch afterwards.
+__device__ __forceinline__ bool consumer_sync_or(int flag) {
+  uint32_t any;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.s32 p, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, 128, p;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(any)
+      : "r"(flag)
+      : "memory");
+  return any != 0;
+}
+
+__device__ __forceinline__ void split_chunks(const DecodeParams& p, int split, int* first,
+                                             int* count) {
+  if (split < p.n - 1) {
+    *first = split * p.nc_full;
+    *count = p.nc_full;
+  } else if (split == p.n - 1) {
+    *first = (p.n - 1) * p.nc_full;
+    *count = p.nc_last;
+  } else {
+    *first = (p.n - 1) * p.nc_full + p.nc_last;
+    *count = p.nc_tail;
+  }
+}
+
 // Reduce the chunk partials of one split (fixed order) into part_o /
-// part_lse. Run by the last CTA that finished a chunk of the split; `sw` is
-// free shared memory (>= kDecRows * (kMaxChunksPerSplit + 2) floats).
+// part_lse. Run by the consumer warps of the CTA that finished the split's
+// last chunk; `sw` is free shared memory of kDecRows * (kMaxChunksPerSplit + 2)
+// floats.
 template <int D>
 __device__ void reduce_split(const DecodeParams& p, int bh, int split, float* sw) {
-  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int nwarps = blockDim.x / 32;
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  constexpr int kC = kMaxChunksPerSplit;
   const int nsplit = p.n + 1;
   int first, count;
-  if (split < p.n - 1) {
-    first = split * p.nc_full;
-    count = p.nc_full;
-  } else if (split == p.n - 1) {
-    first = (p.n - 1) * p.nc_full;
-    count = p.nc_last;
-  } else {
-    first = (p.n - 1) * p.nc_full + p.nc_last;
-    count = p.nc_tail;
-  }
+  split_chunks(p, split, &first, &count);
   const size_t cbase = static_cast<size_t>(bh) * p.chunks_per_head + first;
-  float* wgt = sw;                          // [R][count] weights exp(lse_c - M)
-  float* rowz = sw + kDecRows * kMaxChunksPerSplit;  // [R] sum of weights
-  float* rowm = rowz + kDecRows;            // [R] max statistic
-  for (int rho = warp; rho < p.R; rho += nwarps) {
+  float* wgt = sw;                // [R][kC] weights exp(lse_c - M)
+  float* rowz = sw + kDecRows * kC;  // [R] sum of weights
+  float* rowm = rowz + kDecRows;  // [R] max statistic
+  for (int rho = warp; rho < p.R; rho += kConsumers / 32) {
     float M = -INFINITY;
     for (int c = lane; c < count; c += 32) M = fmaxf(M, p.ws_lse[(cbase + c) * kDecRows + rho]);
 #pragma unroll
@@ -128,7 +155,7 @@ __device__ void reduce_split(const DecodeParams& p, int bh, int split, float* sw
     for (int c = lane; c < count; c += 32) {
       const float l = p.ws_lse[(cbase + c) * kDecRows + rho];
       const float wv = (M == -INFINITY || l == -INFINITY) ? 0.f : expf(l - M);
-      wgt[rho * kMaxChunksPerSplit + c] = wv;
+      wgt[rho * kC + c] = wv;
       z += wv;
     }
 #pragma unroll
@@ -138,44 +165,141 @@ __device__ void reduce_split(const DecodeParams& p, int bh, int split, float* sw
       rowm[rho] = M;
     }
   }
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < p.R * D; idx += blockDim.x) {
-    const int rho = idx / D, d = idx % D;
-    float acc = 0.f;
-    for (int c = 0; c < count; ++c)  // independent loads: the weights are known
-      acc += wgt[rho * kMaxChunksPerSplit + c] * p.ws_o[((cbase + c) * kDecRows + rho) * D + d];
+  consumer_sync();
+  // 4 columns per thread; the chunk loads of a group of 16 are all issued
+  // before any is used (the reduction is latency-bound)
+  for (int idx = tid; idx < p.R * (D / 4); idx += kConsumers) {
+    const int rho = idx / (D / 4), d4 = idx % (D / 4);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int c0 = 0; c0 < count; c0 += 16) {
+      float4 v[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        v[j] = (c0 + j < count)
+                   ? reinterpret_cast<const float4*>(p.ws_o + ((cbase + c0 + j) * kDecRows + rho) * D)[d4]
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const float wv = (c0 + j < count) ? wgt[rho * kC + c0 + j] : 0.f;
+        acc.x += wv * v[j].x;
+        acc.y += wv * v[j].y;
+        acc.z += wv * v[j].z;
+        acc.w += wv * v[j].w;
+      }
+    }
     const float z = rowz[rho];
+    const float inv = (z > 0.f) ? 1.f / z : 0.f;
     const int t = rho / p.g, h = (bh % p.Hkv) * p.g + rho % p.g;
     const int b = bh / p.Hkv;
     const size_t row = ((static_cast<size_t>(b) * p.Hq + h) * nsplit + split) * p.T + t;
-    p.part_o[row * D + d] = (z > 0.f) ? acc / z : 0.f;
-    if (d == 0) p.part_lse[row] = (z > 0.f) ? rowm[rho] + logf(z) : -INFINITY;
+    reinterpret_cast<float4*>(p.part_o + row * D)[d4] =
+        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    if (d4 == 0) p.part_lse[row] = (z > 0.f) ? rowm[rho] + logf(z) : -INFINITY;
   }
 }
 
+// Exact LSE merge of the n+1 split partials of one (batch, KV head) into
+// o_merged / lse_merged: m = max lse_s, w_s = exp(lse_s - m),
+// o = sum w_s o_s / sum w_s, lse = m + log(sum w_s). Consumer warps only.
+template <int D>
+__device__ void merge_head(const DecodeParams& p, int bh, float* sw) {
+  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
+  const int nsplit = p.n + 1;
+  const int b = bh / p.Hkv, kvh = bh % p.Hkv;
+  float* rowm = sw;             // [R]
+  float* rowz = sw + kDecRows;  // [R]
+  auto prow = [&](int rho, int sp) {  // row index into part_o / part_lse
+    const int t = rho / p.g, h = kvh * p.g + rho % p.g;
+    return ((static_cast<size_t>(b) * p.Hq + h) * nsplit + sp) * p.T + t;
+  };
+  for (int rho = warp; rho < p.R; rho += kConsumers / 32) {
+    float M = -INFINITY;
+    for (int sp = lane; sp < nsplit; sp += 32) M = fmaxf(M, p.part_lse[prow(rho, sp)]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float z = 0.f;
+    for (int sp = lane; sp < nsplit; sp += 32) {
+      const float l = p.part_lse[prow(rho, sp)];
+      z += (M == -INFINITY || l == -INFINITY) ? 0.f : expf(l - M);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
+    if (lane == 0) {
+      rowm[rho] = M;
+      rowz[rho] = z;
+    }
+  }
+  consumer_sync();
+  for (int idx = tid; idx < p.R * (D / 4); idx += kConsumers) {
+    const int rho = idx / (D / 4), d4 = idx % (D / 4);
+    const float M = rowm[rho], z = rowz[rho];
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (z > 0.f) {
+      for (int s0 = 0; s0 < nsplit; s0 += 8) {
+        float4 v[8];
+        float wv[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int sp = s0 + j;
+          const float l = (sp < nsplit) ? p.part_lse[prow(rho, sp)] : -INFINITY;
+          wv[j] = (l == -INFINITY) ? 0.f : expf(l - M);
+          v[j] = (sp < nsplit) ? reinterpret_cast<const float4*>(p.part_o + prow(rho, sp) * D)[d4]
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          acc.x += wv[j] * v[j].x;
+          acc.y += wv[j] * v[j].y;
+          acc.z += wv[j] * v[j].z;
+          acc.w += wv[j] * v[j].w;
+        }
+      }
+    }
+    const float inv = (z > 0.f) ? 1.f / z : 0.f;
+    const int t = rho / p.g, h = kvh * p.g + rho % p.g;
+    __nv_bfloat16* dst = p.o_merged + ((static_cast<size_t>(b) * p.T + t) * p.Hq + h) * D + 4 * d4;
+    uint2 pk;
+    pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
+    pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(dst) = pk;
+    if (d4 == 0 && p.lse_merged)
+      p.lse_merged[(static_cast<size_t>(b) * p.Hq + h) * p.T + t] = (z > 0.f) ? M + logf(z) : -INFINITY;
+  }
+}
+
+// Persistent split-KV decode. CTA c owns the contiguous unit range
+// [c*U/G, (c+1)*U/G) of the U = B*Hkv*chunks_per_head (head, chunk) units.
+// The producer warp streams every tile of every unit through one ring; the
+// consumers keep the running softmax of a unit in registers, combine the four
+// warps through shared memory at its end, publish the chunk partial, and the
+// CTA completing a split (or a head) reduces (merges) it while the producer
+// already streams the next unit.
 template <int D>
 __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_constant__ DecodeParams p) {
   constexpr int kHalfBytes = kDecTile * 128;        // one 64-column TMA box of a tile
   constexpr int kTileBytes = kHalfBytes * (D / 64);  // K (or V) tile of 64 keys
   constexpr int kKSteps = D / 16;
+  constexpr int kCombCols = 32;                      // columns combined per round
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                            ~static_cast<uintptr_t>(1023));
   uint8_t* sK = sm;
   uint8_t* sV = sm + kDecStages * kTileBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sm + 2 * kDecStages * kTileBytes);
+  float* comb = reinterpret_cast<float*>(sm + 2 * kDecStages * kTileBytes);  // combine buffer
+  float* cm = comb;                                  // [4][16] warp maxima
+  float* cl = cm + 4 * kDecRows;                     // [4][16] warp sums
+  float* co = cl + 4 * kDecRows;                     // [4][16][kCombCols] warp outputs
+  uint64_t* full = reinterpret_cast<uint64_t*>(co + 4 * kDecRows * kCombCols);
   uint64_t* empty = full + kDecStages;
   __shared__ volatile int abort_flag;
   __shared__ int issued;
+  __shared__ int flag_last;
 
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int unit = blockIdx.x;
-  const int bh = unit / p.chunks_per_head;  // b * Hkv + kvh
-  const int cidx = unit % p.chunks_per_head;
-  const int b = bh / p.Hkv, kvh = bh % p.Hkv;
-  const ChunkRange cr = chunk_range(p, cidx);
-  const int ntiles = ceil_div(cr.k_hi - cr.k_lo, kDecTile);
+  const int units = p.B * p.Hkv * p.chunks_per_head;
+  const int u_begin = static_cast<int>(static_cast<long long>(blockIdx.x) * units / gridDim.x);
+  const int u_end = static_cast<int>(static_cast<long long>(blockIdx.x + 1) * units / gridDim.x);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kDecStages; ++s) {
@@ -188,217 +312,245 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
   }
   __syncthreads();
 
-  // per-thread softmax state (consumer warps)
-  float o[D / 8][4];
-  float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-  const int gq = lane >> 2, t4 = lane & 3;
-  const int r0 = gq, r1 = gq + 8;
-
   if (warp == 4) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       prefetch_tmap(&p.tmK);
       prefetch_tmap(&p.tmV);
-      int it = 0;
-      for (; it < ntiles; ++it) {
-        const int st = it % kDecStages, use = it / kDecStages;
-        if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, &abort_flag, p.status)) break;
-        const int key0 = cr.k_lo + it * kDecTile;
-        mbar_arrive_expect_tx(&full[st], 2 * kTileBytes);
+      int gt = 0;  // tiles issued over all units of this CTA
+      bool stop = false;
+      for (int u = u_begin; u < u_end && !stop; ++u) {
+        const int bh = u / p.chunks_per_head;
+        const ChunkRange cr = chunk_range(p, u % p.chunks_per_head);
+        const int nt = ceil_div(cr.k_hi - cr.k_lo, kDecTile);
+        for (int it = 0; it < nt; ++it, ++gt) {
+          const int st = gt % kDecStages, use = gt / kDecStages;
+          if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, &abort_flag, p.status)) {
+            stop = true;
+            break;
+          }
+          const int key0 = cr.k_lo + it * kDecTile;
+          mbar_arrive_expect_tx(&full[st], 2 * kTileBytes);
 #pragma unroll
-        for (int hd = 0; hd < D / 64; ++hd) {
-          tma_load_3d(sK + st * kTileBytes + hd * kHalfBytes, &p.tmK, &full[st], hd * 64, key0, bh);
-          tma_load_3d(sV + st * kTileBytes + hd * kHalfBytes, &p.tmV, &full[st], hd * 64, key0, bh);
+          for (int hd = 0; hd < D / 64; ++hd) {
+            tma_load_3d(sK + st * kTileBytes + hd * kHalfBytes, &p.tmK, &full[st], hd * 64, key0, bh);
+            tma_load_3d(sV + st * kTileBytes + hd * kHalfBytes, &p.tmV, &full[st], hd * 64, key0, bh);
+          }
         }
       }
-      issued = it;
+      issued = gt;
+      if (abort_flag) {  // let copies still in flight land before the CTA exits
+        for (int it = imax(0, gt - kDecStages); it < gt; ++it)
+          mbar_drain(&full[it % kDecStages], (it / kDecStages) & 1, 100000000ull);
+      }
     }
   } else {
     // ------------------------------------------------------------ consumers
+    const int gq = lane >> 2, t4 = lane & 3;
+    const int r0 = gq, r1 = gq + 8;
     const int g = p.g;
-    // rows rho = t * g + hh of this GQA group; rows >= R are zero padding
-    auto qrow = [&](int rho) -> const __nv_bfloat16* {
-      if (rho >= p.R) return nullptr;
-      int t = rho / g, hh = rho % g;
-      return p.q + ((static_cast<size_t>(b) * p.T + t) * p.Hq + kvh * g + hh) * D;
-    };
-    const __nv_bfloat16* q0 = qrow(r0);
-    const __nv_bfloat16* q1 = qrow(r1);
-    uint32_t qf[kKSteps][4];
-#pragma unroll
-    for (int kk = 0; kk < kKSteps; ++kk) {
-      const int c0 = 16 * kk + 2 * t4;
-      qf[kk][0] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + c0) : 0u;
-      qf[kk][1] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + c0) : 0u;
-      qf[kk][2] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + c0 + 8) : 0u;
-      qf[kk][3] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + c0 + 8) : 0u;
-    }
-#pragma unroll
-    for (int dn = 0; dn < D / 8; ++dn) o[dn][0] = o[dn][1] = o[dn][2] = o[dn][3] = 0.f;
-    const int pos0 = p.L + p.tail_len + r0 / g;  // query positions of this thread's rows
-    const int pos1 = p.L + p.tail_len + r1 / g;
     const float c = p.scale_log2;
-
-    for (int it = 0; it < ntiles; ++it) {
-      const int st = it % kDecStages;
-      if (!mbar_wait(&full[st], (it / kDecStages) & 1, &abort_flag, p.status)) break;
-      const uint32_t kb = smem_u32(sK + st * kTileBytes);
-      const uint32_t vb = smem_u32(sV + st * kTileBytes);
-
-      // S = Q K^T for this warp's 16 keys (two n-tiles of 8 keys)
-      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      {
-        const int key_row = 16 * warp + ((lane >> 4) & 1) * 8 + (lane & 7);
+    uint32_t qf[kKSteps][4];
+    int q_bh = -1;
+    int gt = 0;  // tiles consumed over all units of this CTA
+    for (int u = u_begin; u < u_end; ++u) {
+      const int bh = u / p.chunks_per_head;
+      const int cidx = u % p.chunks_per_head;
+      const int b = bh / p.Hkv, kvh = bh % p.Hkv;
+      const ChunkRange cr = chunk_range(p, cidx);
+      const int nt = ceil_div(cr.k_hi - cr.k_lo, kDecTile);
+      if (bh != q_bh) {  // rows rho = t * g + hh of this GQA group; rows >= R are padding
+        auto qrow = [&](int rho) -> const __nv_bfloat16* {
+          if (rho >= p.R) return nullptr;
+          return p.q + ((static_cast<size_t>(b) * p.T + rho / g) * p.Hq + kvh * g + rho % g) * D;
+        };
+        const __nv_bfloat16* q0 = qrow(r0);
+        const __nv_bfloat16* q1 = qrow(r1);
 #pragma unroll
         for (int kk = 0; kk < kKSteps; ++kk) {
-          const int chunk = 2 * kk + ((lane >> 3) & 1);
-          const uint32_t addr = kb + (chunk >> 3) * kHalfBytes + sw128_offset(key_row, chunk & 7);
-          uint32_t b0, b1, b2, b3;
-          ldsm_x4(addr, b0, b1, b2, b3);
-          mma_16816(s[0], qf[kk], b0, b1);
-          mma_16816(s[1], qf[kk], b2, b3);
+          const int c0 = 16 * kk + 2 * t4;
+          qf[kk][0] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + c0) : 0u;
+          qf[kk][1] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + c0) : 0u;
+          qf[kk][2] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + c0 + 8) : 0u;
+          qf[kk][3] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + c0 + 8) : 0u;
         }
+        q_bh = bh;
       }
-      // visibility: keys [k_lo, k_hi) of this chunk, causal in the tail
-      const int kbase = cr.k_lo + it * kDecTile + 16 * warp + 2 * t4;
+      float o[D / 8][4];
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int key = kbase + 8 * nt + (j & 1);
-          const int pos = (j < 2) ? pos0 : pos1;
-          const bool vis = key < cr.k_hi && (!cr.causal || key <= pos);
-          if (!vis) s[nt][j] = -INFINITY;
-        }
-      // online softmax over the two rows this thread touches
-      float mt0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-      float mt1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-      mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, 1));
-      mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, 2));
-      mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, 1));
-      mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, 2));
-      const float mn0 = fmaxf(m0, mt0), mn1 = fmaxf(m1, mt1);
-      const float a0 = (mn0 == -INFINITY) ? 1.f : ex2_approx((m0 - mn0) * c);
-      const float a1 = (mn1 == -INFINITY) ? 1.f : ex2_approx((m1 - mn1) * c);
-      const float ref0 = (mn0 == -INFINITY) ? 0.f : mn0 * c;
-      const float ref1 = (mn1 == -INFINITY) ? 0.f : mn1 * c;
-      m0 = mn0;
-      m1 = mn1;
-      float pr[2][4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        pr[nt][0] = ex2_approx(fmaf(s[nt][0], c, -ref0));
-        pr[nt][1] = ex2_approx(fmaf(s[nt][1], c, -ref0));
-        pr[nt][2] = ex2_approx(fmaf(s[nt][2], c, -ref1));
-        pr[nt][3] = ex2_approx(fmaf(s[nt][3], c, -ref1));
-      }
-      l0 = l0 * a0 + (pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1]);
-      l1 = l1 * a1 + (pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3]);
-#pragma unroll
-      for (int dn = 0; dn < D / 8; ++dn) {
-        o[dn][0] *= a0;
-        o[dn][1] *= a0;
-        o[dn][2] *= a1;
-        o[dn][3] *= a1;
-      }
-      uint32_t pa[4];
-      pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
-      pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
-      pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
-      pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
-      // O += P V over this warp's 16 keys, two 8-wide d tiles per ldmatrix
-      {
-        const int mi = lane >> 3;
-        const int key_row = 16 * warp + (mi & 1) * 8 + (lane & 7);
-#pragma unroll
-        for (int dn2 = 0; dn2 < D / 16; ++dn2) {
-          const int chunk = 2 * dn2 + (mi >> 1);
-          const uint32_t addr = vb + (chunk >> 3) * kHalfBytes + sw128_offset(key_row, chunk & 7);
-          uint32_t v0, v1, v2, v3;
-          ldsm_x4_t(addr, v0, v1, v2, v3);
-          mma_16816(o[2 * dn2], pa, v0, v1);
-          mma_16816(o[2 * dn2 + 1], pa, v2, v3);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[st]);
-    }
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-  }
+      for (int dn = 0; dn < D / 8; ++dn) o[dn][0] = o[dn][1] = o[dn][2] = o[dn][3] = 0.f;
+      float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+      const int pos0 = p.L + p.tail_len + r0 / g;  // query positions of this thread's rows
+      const int pos1 = p.L + p.tail_len + r1 / g;
 
-  // Drain: make sure no TMA copy still targets this CTA's shared memory.
-  __syncthreads();
-  if (threadIdx.x == 128 && abort_flag) {
-    for (int it = imax(0, issued - kDecStages); it < issued; ++it)
-      mbar_drain(&full[it % kDecStages], (it / kDecStages) & 1, 100000000ull);
-  }
-  __syncthreads();
-  if (abort_flag) return;
-
-  // Combine the 4 warps' partials through shared memory (the ring is free).
-  float* cm = reinterpret_cast<float*>(sm);  // [4][16]
-  float* cl = cm + 4 * kDecRows;             // [4][16]
-  float* co = cl + 4 * kDecRows;             // [4][16][D]
-  if (warp < 4) {
-    if (t4 == 0) {
-      cm[warp * kDecRows + r0] = m0;
-      cm[warp * kDecRows + r1] = m1;
-      cl[warp * kDecRows + r0] = l0;
-      cl[warp * kDecRows + r1] = l1;
-    }
+      for (int it = 0; it < nt; ++it, ++gt) {
+        const int st = gt % kDecStages;
+        if (!mbar_wait(&full[st], (gt / kDecStages) & 1, &abort_flag, p.status)) break;
+        const uint32_t kb = smem_u32(sK + st * kTileBytes);
+        const uint32_t vb = smem_u32(sV + st * kTileBytes);
+        // S = Q K^T for this warp's 16 keys (two n-tiles of 8 keys)
+        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        {
+          const int key_row = 16 * warp + ((lane >> 4) & 1) * 8 + (lane & 7);
 #pragma unroll
-    for (int dn = 0; dn < D / 8; ++dn) {
-      const int d = 8 * dn + 2 * t4;
-      co[(warp * kDecRows + r0) * D + d] = o[dn][0];
-      co[(warp * kDecRows + r0) * D + d + 1] = o[dn][1];
-      co[(warp * kDecRows + r1) * D + d] = o[dn][2];
-      co[(warp * kDecRows + r1) * D + d + 1] = o[dn][3];
-    }
-  }
-  __syncthreads();
-  const size_t base = static_cast<size_t>(bh) * p.chunks_per_head + cidx;
-  for (int idx = threadIdx.x; idx < p.R * D; idx += blockDim.x) {
-    const int rho = idx / D, d = idx % D;
-    float M = -INFINITY;
+          for (int kk = 0; kk < kKSteps; ++kk) {
+            const int chunk = 2 * kk + ((lane >> 3) & 1);
+            const uint32_t addr = kb + (chunk >> 3) * kHalfBytes + sw128_offset(key_row, chunk & 7);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(addr, b0, b1, b2, b3);
+            mma_16816(s[0], qf[kk], b0, b1);
+            mma_16816(s[1], qf[kk], b2, b3);
+          }
+        }
+        // visibility: keys [k_lo, k_hi) of this chunk, causal in the tail
+        const int kbase = cr.k_lo + it * kDecTile + 16 * warp + 2 * t4;
 #pragma unroll
-    for (int w = 0; w < 4; ++w) M = fmaxf(M, cm[w * kDecRows + rho]);
-    float out = 0.f, lse = -INFINITY;
-    if (M != -INFINITY) {
-      float Ls = 0.f, acc = 0.f;
+        for (int ntl = 0; ntl < 2; ++ntl)
 #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        const float e = ex2_approx((cm[w * kDecRows + rho] - M) * p.scale_log2);
-        Ls += e * cl[w * kDecRows + rho];
-        acc += e * co[(w * kDecRows + rho) * D + d];
+          for (int j = 0; j < 4; ++j) {
+            const int key = kbase + 8 * ntl + (j & 1);
+            const int pos = (j < 2) ? pos0 : pos1;
+            const bool vis = key < cr.k_hi && (!cr.causal || key <= pos);
+            if (!vis) s[ntl][j] = -INFINITY;
+          }
+        // online softmax over the two rows this thread touches
+        float mt0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+        float mt1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+        mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, 1));
+        mt0 = fmaxf(mt0, __shfl_xor_sync(0xffffffffu, mt0, 2));
+        mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, 1));
+        mt1 = fmaxf(mt1, __shfl_xor_sync(0xffffffffu, mt1, 2));
+        const float mn0 = fmaxf(m0, mt0), mn1 = fmaxf(m1, mt1);
+        const float a0 = (mn0 == -INFINITY) ? 1.f : ex2_approx((m0 - mn0) * c);
+        const float a1 = (mn1 == -INFINITY) ? 1.f : ex2_approx((m1 - mn1) * c);
+        const float ref0 = (mn0 == -INFINITY) ? 0.f : mn0 * c;
+        const float ref1 = (mn1 == -INFINITY) ? 0.f : mn1 * c;
+        m0 = mn0;
+        m1 = mn1;
+        float pr[2][4];
+#pragma unroll
+        for (int ntl = 0; ntl < 2; ++ntl) {
+          pr[ntl][0] = ex2_approx(fmaf(s[ntl][0], c, -ref0));
+          pr[ntl][1] = ex2_approx(fmaf(s[ntl][1], c, -ref0));
+          pr[ntl][2] = ex2_approx(fmaf(s[ntl][2], c, -ref1));
+          pr[ntl][3] = ex2_approx(fmaf(s[ntl][3], c, -ref1));
+        }
+        l0 = l0 * a0 + (pr[0][0] + pr[0][1] + pr[1][0] + pr[1][1]);
+        l1 = l1 * a1 + (pr[0][2] + pr[0][3] + pr[1][2] + pr[1][3]);
+#pragma unroll
+        for (int dn = 0; dn < D / 8; ++dn) {
+          o[dn][0] *= a0;
+          o[dn][1] *= a0;
+          o[dn][2] *= a1;
+          o[dn][3] *= a1;
+        }
+        uint32_t pa[4];
+        pa[0] = pack_bf16x2(pr[0][0], pr[0][1]);
+        pa[1] = pack_bf16x2(pr[0][2], pr[0][3]);
+        pa[2] = pack_bf16x2(pr[1][0], pr[1][1]);
+        pa[3] = pack_bf16x2(pr[1][2], pr[1][3]);
+        // O += P V over this warp's 16 keys, two 8-wide d tiles per ldmatrix
+        {
+          const int mi = lane >> 3;
+          const int key_row = 16 * warp + (mi & 1) * 8 + (lane & 7);
+#pragma unroll
+          for (int dn2 = 0; dn2 < D / 16; ++dn2) {
+            const int chunk = 2 * dn2 + (mi >> 1);
+            const uint32_t addr = vb + (chunk >> 3) * kHalfBytes + sw128_offset(key_row, chunk & 7);
+            uint32_t v0, v1, v2, v3;
+            ldsm_x4_t(addr, v0, v1, v2, v3);
+            mma_16816(o[2 * dn2], pa, v0, v1);
+            mma_16816(o[2 * dn2 + 1], pa, v2, v3);
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[st]);
       }
-      out = acc / Ls;
-      lse = M * p.scale_ln + logf(Ls);
+      // all four consumer warps decide together whether to stop (a warp still
+      // inside the tile loop would otherwise miss the named barriers below)
+      if (consumer_sync_or(abort_flag)) break;
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+      l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+      l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+
+      // ---- combine the four warps' partials, kCombCols columns per round
+      const size_t base = static_cast<size_t>(bh) * p.chunks_per_head + cidx;
+      if (t4 == 0) {
+        cm[warp * kDecRows + r0] = m0;
+        cm[warp * kDecRows + r1] = m1;
+        cl[warp * kDecRows + r0] = l0;
+        cl[warp * kDecRows + r1] = l1;
+      }
+#pragma unroll
+      for (int rd = 0; rd < D / kCombCols; ++rd) {
+#pragma unroll
+        for (int dn = rd * (kCombCols / 8); dn < (rd + 1) * (kCombCols / 8); ++dn) {
+          const int d = 8 * dn + 2 * t4 - rd * kCombCols;
+          co[(warp * kDecRows + r0) * kCombCols + d] = o[dn][0];
+          co[(warp * kDecRows + r0) * kCombCols + d + 1] = o[dn][1];
+          co[(warp * kDecRows + r1) * kCombCols + d] = o[dn][2];
+          co[(warp * kDecRows + r1) * kCombCols + d + 1] = o[dn][3];
+        }
+        consumer_sync();
+        for (int idx = threadIdx.x; idx < p.R * kCombCols; idx += kConsumers) {
+          const int rho = idx / kCombCols, dc = idx % kCombCols;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) M = fmaxf(M, cm[w * kDecRows + rho]);
+          float out = 0.f, lse = -INFINITY;
+          if (M != -INFINITY) {
+            float Ls = 0.f, acc = 0.f;
+#pragma unroll
+            for (int w = 0; w < 4; ++w) {
+              const float e = ex2_approx((cm[w * kDecRows + rho] - M) * c);
+              Ls += e * cl[w * kDecRows + rho];
+              acc += e * co[(w * kDecRows + rho) * kCombCols + dc];
+            }
+            out = acc / Ls;
+            lse = M * p.scale_ln + logf(Ls);
+          }
+          p.ws_o[(base * kDecRows + rho) * D + rd * kCombCols + dc] = out;
+          if (rd == 0 && dc == 0) p.ws_lse[base * kDecRows + rho] = lse;
+        }
+        consumer_sync();
+      }
+      // ---- the CTA completing a split reduces it; the one completing a head
+      // merges it. After the consumer barrier one thread publishes the CTA's
+      // writes (fence, then count itself in) and, if last, fences again so
+      // the partials of the other CTAs are visible before anyone reads them.
+      consumer_sync();
+      if (threadIdx.x == 0) {
+        int first, count;
+        split_chunks(p, cr.split, &first, &count);
+        __threadfence();
+        flag_last = (atomicAdd(&p.counters[bh * (p.n + 1) + cr.split], 1) == count - 1);
+        __threadfence();
+      }
+      consumer_sync();
+      if (flag_last) {
+        reduce_split<D>(p, bh, cr.split, comb);
+        consumer_sync();
+        if (p.o_merged != nullptr) {
+          if (threadIdx.x == 0) {
+            __threadfence();
+            flag_last = (atomicAdd(&p.head_counters[bh], 1) == p.n);
+            __threadfence();
+          }
+          consumer_sync();
+          if (flag_last) merge_head<D>(p, bh, comb);
+          consumer_sync();
+        }
+      }
     }
-    p.ws_o[(base * kDecRows + rho) * D + d] = out;
-    if (d == 0) p.ws_lse[base * kDecRows + rho] = lse;
-  }
-  // The last CTA to finish a chunk of this split reduces the split: every
-  // CTA publishes its partial (fence) before counting itself in.
-  __shared__ int is_last;
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    const int prev = atomicAdd(&p.counters[bh * (p.n + 1) + cr.split], 1);
-    const int in_split = cr.split < p.n - 1 ? p.nc_full : (cr.split == p.n - 1 ? p.nc_last : p.nc_tail);
-    is_last = (prev == in_split - 1);
   }
   __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  reduce_split<D>(p, bh, cr.split, reinterpret_cast<float*>(sm));
 }
 
 size_t decode_smem_bytes(int D) {
   const size_t tile = static_cast<size_t>(kDecTile) * D * 2;
-  return 1024 + 2 * kDecStages * tile + 2 * kDecStages * sizeof(uint64_t);
+  const size_t comb = (2 * 4 * kDecRows + 4 * kDecRows * 32) * sizeof(float);
+  return 1024 + 2 * kDecStages * tile + comb + 2 * kDecStages * sizeof(uint64_t);
 }
 
 cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t stream) {
@@ -415,10 +567,13 @@ cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     if (dev < 64) attr[dev] = true;
   }
+  int sms = 148;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = imin(units, 2 * sms);  // persistent: two CTAs per SM
   if (D == 128)
-    decode_kernel<128><<<units, kDecThreads, smem, stream>>>(p);
+    decode_kernel<128><<<grid, kDecThreads, smem, stream>>>(p);
   else
-    decode_kernel<64><<<units, kDecThreads, smem, stream>>>(p);
+    decode_kernel<64><<<grid, kDecThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

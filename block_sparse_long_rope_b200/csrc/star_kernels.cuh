@@ -55,7 +55,7 @@ cudaError_t launch_attn(const AttnParams& p, int D, cudaStream_t stream);
 // ---- Phase 2 decode (split-KV, HBM-bound) ----------------------------------
 constexpr int kDecRows = 16;   // (token, head) rows per CTA: one mma.sync M tile
 constexpr int kDecTile = 64;   // keys per staged K/V tile
-constexpr int kMaxChunksPerSplit = 16;  // chunk size is chosen so a split has at most this many
+constexpr int kMaxChunksPerSplit = 64;  // chunk size is chosen so a split has at most this many
 struct DecodeParams {
   CUtensorMap tmK;  // K cache: dims {D, Lvalid, B*Hkv}, box {64, 64, 1}
   CUtensorMap tmV;
@@ -67,6 +67,9 @@ struct DecodeParams {
   float* ws_o;     // [B*Hkv, chunks_per_head, kDecRows, D] chunk-normalised output
   float* ws_lse;   // [B*Hkv, chunks_per_head, kDecRows]
   int* counters;   // [B*Hkv, n+1] finished chunks per split, zero at launch
+  int* head_counters;  // [B*Hkv] finished splits per (batch, KV head), zero at launch
+  __nv_bfloat16* o_merged;  // nullable: [B, T, Hq, D] merged output (also needs head_counters)
+  float* lse_merged;        // nullable: [B, Hq, T]
   float* part_o;   // [B, Hq, n+1, T, D]
   float* part_lse; // [B, Hq, n+1, T]
   int* status;

@@ -73,7 +73,21 @@ class StarLayer:
         return po, pl
 
     def attend(self, q, k, v, tail_len):
-        """Partials then merge: returns (o[B,T,Hq,D] bf16, lse[B,Hq,T])."""
+        """Partials and their exact merge in one call (star_phase2_attend):
+        returns (o[B,T,Hq,D] bf16, lse[B,Hq,T]) views of the layer's buffers."""
+        b = self.buf
+        B, T, Hq, D = q.shape
+        S = b.part_o.shape[2]
+        po = _prefix_view(b.part_o, (B, Hq, S, T, D))
+        pl = _prefix_view(b.part_lse, (B, Hq, S, T))
+        o = _prefix_view(b.o2, (B, T, Hq, D))
+        lse = _prefix_view(b.lse2, (B, Hq, T))
+        star.star_phase2_attend(q, k, v, b.k_cache, b.v_cache, self.w.L, self.w.block_len,
+                                tail_len, po, pl, o, self.w.theta, b.ws2, lse=lse)
+        return o, lse
+
+    def attend_unfused(self, q, k, v, tail_len):
+        """star_phase2_partial then star_lse_merge (two calls)."""
         po, pl = self.partial(q, k, v, tail_len)
         B, Hq, S, T, D = po.shape
         o = _prefix_view(self.buf.o2, (B, T, Hq, D))

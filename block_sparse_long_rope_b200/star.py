@@ -102,6 +102,27 @@ def star_phase2_partial(q, k, v, k_cache, v_cache, L, block_len, tail_len, part_
     return ns.value
 
 
+def star_phase2_attend(q, k, v, k_cache, v_cache, L, block_len, tail_len, part_o, part_lse, o,
+                       theta, workspace, lse=None, stream=None):
+    """star_phase2_partial plus the exact merge in one call: writes the
+    partials and o[B,T,Hq,D] bf16 / lse[B,Hq,T] (optional). Returns nsplit."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (k_cache, "k_cache"), (v_cache, "v_cache"), (o, "o")):
+        _bf16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    B, T, Hq, D = q.shape
+    Hkv = k.shape[2]
+    Lcap = k_cache.shape[2]
+    ns = ctypes.c_int(0)
+    lib = _abi.load()
+    _abi.check(lib.star_phase2_attend(
+        _ptr(q), _ptr(k), _ptr(v), T, _ptr(k_cache), _ptr(v_cache), Lcap, int(L), int(block_len),
+        int(tail_len), _ptr(part_o), _ptr(part_lse), _ptr(o), _ptr(lse), ctypes.byref(ns), B, Hq,
+        Hkv, D, float(theta), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return ns.value
+
+
 def star_phase2_decode_static(q, k, v, k_cache, v_cache, L, block_len, tail_len, part_o,
                               part_lse, theta, stream=None):
     """star_phase2_partial for decode steps without a workspace: the scratch

@@ -143,6 +143,22 @@ star_status star_phase2_partial(const void* q, const void* k, const void* v, int
                                 size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * star_phase2_attend — star_phase2_partial followed by the exact merge of its
+ * partials (as star_lse_merge) in the same call [pith 2WVXFXZ2, Referee
+ * summary; minor comment on Algorithm 2]. part_o / part_lse are written as
+ * by star_phase2_partial; o[B, T, Hq, D] bf16 (required) and lse[B, Hq, T]
+ * fp32 (nullable) receive the merged global attention. On the decode path
+ * (T * Hq / Hkv <= 16) the merge runs inside the decode kernel: the last CTA
+ * to finish the splits of a (batch, KV head) merges them, so no extra launch
+ * is made. Workspace as for star_phase2_partial.
+ */
+star_status star_phase2_attend(const void* q, const void* k, const void* v, int T, void* k_cache,
+                               void* v_cache, int Lcap, int L, int block_len, int tail_len,
+                               float* part_o, float* part_lse, void* o, float* lse,
+                               int* nsplit_out, int B, int Hq, int Hkv, int D, double theta,
+                               void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * star_lse_merge — exact merge of per-split partials into global attention
  * [pith 2WVXFXZ2, minor comment on Algorithm 2 (corrected update
  * exp(s_h - s_global) * A_h); assumptions: online softmax aggregation gives

@@ -90,6 +90,20 @@ def run_flow(B, L, Hq, Hkv, D, b, a, theta, Ts, seed):
             gl2.append(l_)
         assert max_abs(go, np.concatenate(go2)) <= TOL_O
         assert max_abs(gl, np.concatenate(gl2)) <= TOL_LSE
+        # the fused call (partials + in-call merge) gives the same merged result;
+        # it rewrites the same appended cache rows with identical values
+        po2 = torch.full_like(po, float("nan"))
+        pl2 = torch.full_like(pl, float("nan"))
+        om2 = torch.full_like(om, float("nan"))
+        lm2 = torch.full_like(lm, float("nan"))
+        ns2 = star.star_phase2_attend(qt, kt, vt, kc, vc, L, b, tail, po2, pl2, om2, theta, ws,
+                                      lse=lm2)
+        star.star_device_status(ws)
+        torch.cuda.synchronize()
+        assert ns2 == n + 1
+        assert max_abs(to64(om2).transpose(0, 2, 1, 3).reshape(-1, D), mo) <= TOL_O
+        assert max_abs(to64(lm2).reshape(-1), ml) <= TOL_LSE
+        assert torch.equal(po2, po) and torch.equal(pl2, pl)
         # the appended cache rows hold the rotated new keys
         kref = orc.rope(kt.cpu(), np.arange(L + tail, L + tail + T), theta, round_out=True)
         kgot = to64(kc[:, :, L + tail:L + tail + T]).transpose(0, 2, 1, 3)
@@ -111,3 +125,31 @@ FLOWS = [
 def test_phase2_flow_matches_oracle(flow):
     B, L, Hq, Hkv, D, b, a, theta, Ts = flow
     run_flow(B, L, Hq, Hkv, D, b, a, theta, Ts, seed=L)
+
+
+def test_graph_replay_matches_eager_step():
+    """A full layer step captured as a CUDA graph and replayed reproduces the
+    eager step bit for bit (all launches are deterministic)."""
+    from block_sparse_long_rope_b200 import inputs
+    from block_sparse_long_rope_b200.configs import WORKLOADS
+    from block_sparse_long_rope_b200.pipeline import StarLayer, phase2_calls
+
+    w = WORKLOADS[0]
+    ctx = inputs.make_context(w.B, w.L, w.Hq, w.Hkv, w.D, w.index, device="cuda")
+    new = inputs.make_new_tokens(w.B, w.Tq + w.Tdec, w.Hq, w.Hkv, w.D, w.index, device="cuda")
+    calls = phase2_calls(w, *new)
+    layer = StarLayer(w)
+    o_e, lse_e = layer.step(ctx, calls)
+    ref = (layer.buf.o.clone(), layer.buf.lse.clone(), o_e.clone(), lse_e.clone())
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        o_g, lse_g = layer.step(ctx, calls)
+    layer.buf.o.zero_()
+    o_g.zero_()
+    g.replay()
+    g.replay()
+    star.star_device_status(layer.buf.ws2)
+    torch.cuda.synchronize()
+    assert torch.equal(layer.buf.o, ref[0]) and torch.equal(layer.buf.lse, ref[1])
+    assert torch.equal(o_g, ref[2]) and torch.equal(lse_g, ref[3])
