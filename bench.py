@@ -136,6 +136,27 @@ def oracle_sample(w, budget_s=15.0, seed=0):
     return est_step, sample, t_p1 + t_dec
 
 
+def phase1_traffic(workload):
+    """DRAM bytes (read + write) of one star_phase1_encode launch from the ncu
+    capture recorded under profiles/, if the kernel sources are still the ones
+    that were profiled; None otherwise (the counters no longer apply)."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", f"phase1_traffic_{workload}.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)
+        h = hashlib.sha256()
+        for src in rec["sources"]:
+            with open(os.path.join(ROOT, src), "rb") as g:
+                h.update(g.read())
+        if h.hexdigest() != rec["sources_sha256"]:
+            return None
+        return int(rec["traffic_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        return None
+
+
 def max_over_ranks(values, device, world):
     """Element-wise max of per-rank timings (ms) over all ranks."""
     if world <= 1:
@@ -350,7 +371,8 @@ def run_star(args, w, rank, world, local_rank):
                      "peak_source": f"{peak_src} bf16_tflops (burst)",
                      "algorithmic": "4*D*Hq*B*[n*b(b+1)/2 + (n-1)*a*b] unmasked FLOPs per launch "
                                     f"= {p1_flops:.4g}",
-                     "traffic": None},
+                     "traffic": phase1_traffic(w.name),
+                     "traffic_unit": "bytes per launch (DRAM read + write, ncu)"},
         "e2e": {"value": round(job_value(w.B * w.L, world, e2e_ms / K), 1), "unit": "tok/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": launches * K,
