@@ -326,7 +326,7 @@ def run_star(args, w, rank, world, local_rank):
     dec_gbs = dec_bytes / dec_s / 1e9 if dec_s > 0 else None
     dec_tok_s = w.B * w.Tdec / dec_s if dec_s > 0 else None
     chunk_s = chunk_ms / K / 1e3
-    launches = 2 + 3 + 2 * w.Tdec  # rope+attn; rope+attn+merge; (rope+decode) x Tdec
+    launches = 2 + 3 + w.Tdec  # rope+attn; rope+attn+merge; one decode kernel per token
 
     line = {
         "metric": METRIC,
@@ -360,8 +360,8 @@ def run_star(args, w, rank, world, local_rank):
             "phase2_decode": {"ms": round(dec_s * 1e3, 4), "tok_s": round(dec_tok_s, 1),
                               "kv_gbs": round(dec_gbs, 1),
                               "frac_hbm": round(dec_gbs / hbm_peak, 4),
-                              "note": "per decode step: RoPE/append kernel + split-KV decode "
-                                      "kernel (split reduce and merge in-kernel); the cache was "
+                              "note": "per decode step: one kernel (RoPE/append, split-KV "
+                                      "decode, split reduce and merge); the cache was "
                                       "just written by Phase 1, so a cache smaller than L2 "
                                       "(126 MB) reads partly from L2"},
         },

@@ -395,7 +395,7 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   if (e != cudaSuccess) return cuda_fail(e, "status reset");
 
   // RoPE of the new tokens at positions L + tail_len + t; K/V appended to the
-  // cache rows of the same index.
+  // cache rows of the same index. The decode kernel does both itself.
   const int row0 = L + tail_len;
   star::RopeParams rp{};
   const long long qs[3] = {(long long)T * Hq * D, (long long)Hq * D, D};
@@ -415,8 +415,10 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   rp.pos = nullptr;
   rp.pos0 = row0;
   star::rope_set_freq(rp, D, theta);
-  e = star::launch_rope(rp, 3, st);
-  if (e != cudaSuccess) return cuda_fail(e, "rope launch");
+  if (!decode) {
+    e = star::launch_rope(rp, 3, st);
+    if (e != cudaSuccess) return cuda_fail(e, "rope launch");
+  }
 
   const int n = ceil_div(L, block_len);
   const int nsplit = n + 1;
@@ -429,7 +431,13 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
     memset(&dp, 0, sizeof dp);
     if ((s = map_cache(&dp.tmK, k_cache, B * Hkv, Lcap, valid, D, star::kDecTile)) != STAR_OK) return s;
     if ((s = map_cache(&dp.tmV, v_cache, B * Hkv, Lcap, valid, D, star::kDecTile)) != STAR_OK) return s;
-    dp.q = qrot;
+    dp.q_new = static_cast<const __nv_bfloat16*>(q);
+    dp.k_new = static_cast<const __nv_bfloat16*>(k);
+    dp.v_new = static_cast<const __nv_bfloat16*>(v);
+    dp.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+    dp.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+    dp.Lcap = Lcap;
+    star::rope_fill_freq(dp.inv_freq, D, theta);
     dp.B = B;
     dp.T = T;
     dp.Hq = Hq;

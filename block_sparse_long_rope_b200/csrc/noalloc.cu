@@ -5,8 +5,8 @@
 // example a plugin whose host application owns every device allocation and
 // exposes only tensors and a stream, or a latency-critical serving loop that
 // must never reach cudaMalloc/cudaFree (they can block and synchronise the
-// device). Such a caller passes its inputs and outputs only; the rotated
-// query and the per-chunk partials of the split-KV decode kernel live in
+// device). Such a caller passes its inputs and outputs only; the split
+// counters and the per-chunk partials of the split-KV decode kernel live in
 // kStaticScratchBytes (16 MiB) of device memory declared below, which every
 // GPU that loads the library holds until the process exits.
 //
@@ -41,7 +41,7 @@ constexpr size_t kStaticScratchBytes = 16u << 20;  // 16 MiB
 constexpr int kMinChunk = 256;
 constexpr int kMaxChunk = 65536;
 
-// The scratch itself: status header | rotated q | chunk outputs | chunk LSEs.
+// The scratch itself: status header and counters | chunk outputs | chunk LSEs.
 static __device__ __align__(256) unsigned char g_scratch[kStaticScratchBytes];
 
 struct DeviceSlot {
@@ -165,11 +165,10 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
   // scratch layout and chunk size: the smallest chunk (>= 256 keys) that both
   // fits the array and leaves several CTAs per SM
   const int n = star::ceil_div(L, block_len);
-  const size_t qrot_bytes = align256((size_t)B * T * Hq * D * 2);
   // zeroed header: status word, then one finished-chunk counter per split
   const size_t zero_bytes = star::kStatusBytes + align256((size_t)B * Hkv * (n + 1) * sizeof(int)) +
                             align256((size_t)B * Hkv * sizeof(int));
-  const size_t head_bytes = zero_bytes + qrot_bytes;
+  const size_t head_bytes = zero_bytes;
   void* base = nullptr;
   int sms = 148;
   star_status st = scratch_address(&base, &sms);
@@ -203,37 +202,20 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
   unsigned char* ws = static_cast<unsigned char*>(base);
   cudaError_t e = cudaMemsetAsync(ws, 0, zero_bytes, stream);
   if (e != cudaSuccess) return fail_static(STAR_ERR_CUDA, "status reset: %s", cudaGetErrorString(e));
-  __nv_bfloat16* qrot = reinterpret_cast<__nv_bfloat16*>(ws + zero_bytes);
-
-  // RoPE of the new tokens; K/V appended to the cache rows L + tail_len + t
-  const int row0 = L + tail_len;
-  star::RopeParams rp{};
-  const long long qs[3] = {(long long)T * Hq * D, (long long)Hq * D, D};
-  const long long ks[3] = {(long long)T * Hkv * D, (long long)Hkv * D, D};
-  const long long cs[3] = {(long long)Hkv * Lcap * D, D, (long long)Lcap * D};
-  rp.job[0] = star::RopeJob{static_cast<const __nv_bfloat16*>(q), qrot, {qs[0], qs[1], qs[2]},
-                            {qs[0], qs[1], qs[2]}, Hq, 1};
-  rp.job[1] = star::RopeJob{static_cast<const __nv_bfloat16*>(k),
-                            static_cast<__nv_bfloat16*>(k_cache) + (size_t)row0 * D,
-                            {ks[0], ks[1], ks[2]}, {cs[0], cs[1], cs[2]}, Hkv, 1};
-  rp.job[2] = star::RopeJob{static_cast<const __nv_bfloat16*>(v),
-                            static_cast<__nv_bfloat16*>(v_cache) + (size_t)row0 * D,
-                            {ks[0], ks[1], ks[2]}, {cs[0], cs[1], cs[2]}, Hkv, 0};
-  rp.B = B;
-  rp.S = T;
-  rp.D = D;
-  rp.pos = nullptr;
-  rp.pos0 = row0;
-  star::rope_set_freq(rp, D, theta);
-  e = star::launch_rope(rp, 3, stream);
-  if (e != cudaSuccess) return fail_static(STAR_ERR_CUDA, "rope launch: %s", cudaGetErrorString(e));
 
   star::DecodeParams dp;
   memset(&dp, 0, sizeof dp);
   const int valid = L + tail_len + T;
   if ((st = cache_map(&dp.tmK, k_cache, B * Hkv, Lcap, valid, D)) != STAR_OK) return st;
   if ((st = cache_map(&dp.tmV, v_cache, B * Hkv, Lcap, valid, D)) != STAR_OK) return st;
-  dp.q = qrot;
+  // the decode kernel rotates q and appends the rotated k and v itself
+  dp.q_new = static_cast<const __nv_bfloat16*>(q);
+  dp.k_new = static_cast<const __nv_bfloat16*>(k);
+  dp.v_new = static_cast<const __nv_bfloat16*>(v);
+  dp.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+  dp.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+  dp.Lcap = Lcap;
+  star::rope_fill_freq(dp.inv_freq, D, theta);
   dp.B = B;
   dp.T = T;
   dp.Hq = Hq;

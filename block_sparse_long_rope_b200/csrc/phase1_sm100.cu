@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                            cc, nref), x0, x1);
           float p0 = 0.f, p1 = 0.f;
           bool on_fma = false;
-          if constexpr (kPolyEvery > 0) on_fma = (j % kPolyEvery) == kPolyEvery - 1;
+          if constexpr (kPolyEvery > 0) on_fma = (j % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
           if (on_fma) {
             p0 = exp2_poly(x0);
             p1 = exp2_poly(x1);

@@ -25,6 +25,7 @@
 //    warp shuffles; per-warp partials are combined through shared memory.
 #include <math.h>
 
+#include "rope_math.cuh"
 #include "star_common.cuh"
 #include "star_kernels.cuh"
 
@@ -317,30 +318,66 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     if (lane == 0) {
       prefetch_tmap(&p.tmK);
       prefetch_tmap(&p.tmV);
-      int gt = 0;  // tiles issued over all units of this CTA
-      bool stop = false;
-      for (int u = u_begin; u < u_end && !stop; ++u) {
-        const int bh = u / p.chunks_per_head;
-        const ChunkRange cr = chunk_range(p, u % p.chunks_per_head);
-        const int nt = ceil_div(cr.k_hi - cr.k_lo, kDecTile);
-        for (int it = 0; it < nt; ++it, ++gt) {
+    }
+    const int row0 = p.L + p.tail_len;  // cache row (= position) of new token 0
+    int gt = 0;  // tiles issued over all units of this CTA
+    bool stop = false;
+    for (int u = u_begin; u < u_end && !stop; ++u) {
+      const int bh = u / p.chunks_per_head;
+      const ChunkRange cr = chunk_range(p, u % p.chunks_per_head);
+      const int nt = ceil_div(cr.k_hi - cr.k_lo, kDecTile);
+      // This call's tokens: the unit whose key range holds a new token's cache
+      // row rotates its key and appends key and value before loading that
+      // tile (no other unit reads the row). The warp writes, every lane
+      // fences its generic writes against the TMA (async proxy) reads.
+      const int w_lo = imax(cr.k_lo, row0), w_hi = imin(cr.k_hi, row0 + p.T);
+      if (w_lo < w_hi) {
+        const int b = bh / p.Hkv, kvh = bh % p.Hkv;
+        for (int r = w_lo; r < w_hi; ++r) {
+          const int t = r - row0;
+          const __nv_bfloat16* ks = p.k_new + ((static_cast<size_t>(b) * p.T + t) * p.Hkv + kvh) * D;
+          const __nv_bfloat16* vs = p.v_new + ((static_cast<size_t>(b) * p.T + t) * p.Hkv + kvh) * D;
+          __nv_bfloat16* kd = p.k_cache + (static_cast<size_t>(bh) * p.Lcap + r) * D;
+          __nv_bfloat16* vd = p.v_cache + (static_cast<size_t>(bh) * p.Lcap + r) * D;
+          for (int i = lane; i < D / 2; i += 32) {
+            double c64, s64;
+            rope_angle(r, p.inv_freq[i], &c64, &s64);
+            const float a = __bfloat162float(ks[i]), bb = __bfloat162float(ks[i + D / 2]);
+            const float c32 = static_cast<float>(c64), s32 = static_cast<float>(s64);
+            kd[i] = __ushort_as_bfloat16(static_cast<unsigned short>(rope_rotate_bf16(a, bb, c32, s32, c64, s64, true)));
+            kd[i + D / 2] = __ushort_as_bfloat16(static_cast<unsigned short>(rope_rotate_bf16(a, bb, c32, s32, c64, s64, false)));
+          }
+          for (int i = lane; i < D; i += 32) vd[i] = vs[i];
+        }
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __syncwarp();
+      }
+      for (int it = 0; it < nt; ++it, ++gt) {
+        int ok = 1;
+        if (lane == 0) {
           const int st = gt % kDecStages, use = gt / kDecStages;
           if (use > 0 && !mbar_wait(&empty[st], (use - 1) & 1, &abort_flag, p.status)) {
-            stop = true;
-            break;
-          }
-          const int key0 = cr.k_lo + it * kDecTile;
-          mbar_arrive_expect_tx(&full[st], 2 * kTileBytes);
+            ok = 0;
+          } else {
+            const int key0 = cr.k_lo + it * kDecTile;
+            mbar_arrive_expect_tx(&full[st], 2 * kTileBytes);
 #pragma unroll
-          for (int hd = 0; hd < D / 64; ++hd) {
-            tma_load_3d(sK + st * kTileBytes + hd * kHalfBytes, &p.tmK, &full[st], hd * 64, key0, bh);
-            tma_load_3d(sV + st * kTileBytes + hd * kHalfBytes, &p.tmV, &full[st], hd * 64, key0, bh);
+            for (int hd = 0; hd < D / 64; ++hd) {
+              tma_load_3d(sK + st * kTileBytes + hd * kHalfBytes, &p.tmK, &full[st], hd * 64, key0, bh);
+              tma_load_3d(sV + st * kTileBytes + hd * kHalfBytes, &p.tmV, &full[st], hd * 64, key0, bh);
+            }
           }
         }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
+          stop = true;
+          break;
+        }
       }
-      issued = gt;
+    }
+    if (lane == 0) {
+      issued = gt;  // a failed wait breaks before counting its tile
       if (abort_flag) {  // let copies still in flight land before the CTA exits
-        for (int it = imax(0, gt - kDecStages); it < gt; ++it)
+        for (int it = imax(0, issued - kDecStages); it < issued; ++it)
           mbar_drain(&full[it % kDecStages], (it / kDecStages) & 1, 100000000ull);
       }
     }
@@ -359,21 +396,38 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
       const int b = bh / p.Hkv, kvh = bh % p.Hkv;
       const ChunkRange cr = chunk_range(p, cidx);
       const int nt = ceil_div(cr.k_hi - cr.k_lo, kDecTile);
-      if (bh != q_bh) {  // rows rho = t * g + hh of this GQA group; rows >= R are padding
-        auto qrow = [&](int rho) -> const __nv_bfloat16* {
-          if (rho >= p.R) return nullptr;
-          return p.q + ((static_cast<size_t>(b) * p.T + rho / g) * p.Hq + kvh * g + rho % g) * D;
-        };
-        const __nv_bfloat16* q0 = qrow(r0);
-        const __nv_bfloat16* q1 = qrow(r1);
+      if (bh != q_bh) {
+        // rows rho = t * g + hh of this GQA group (rows >= R are zero padding):
+        // rotate them here (shared RoPE arithmetic, bit-identical to the
+        // RoPE kernel) into the free combine buffer, then take fragments
+        uint16_t* qs = reinterpret_cast<uint16_t*>(comb);  // [kDecRows][D] bf16 bits
+        for (int e = threadIdx.x; e < kDecRows * (D / 2); e += kConsumers) {
+          const int rho = e / (D / 2), i = e % (D / 2);
+          uint32_t y0 = 0, y1 = 0;
+          if (rho < p.R) {
+            const int t = rho / g, hh = rho % g;
+            const __nv_bfloat16* src =
+                p.q_new + ((static_cast<size_t>(b) * p.T + t) * p.Hq + kvh * g + hh) * D;
+            double c64, s64;
+            rope_angle(p.L + p.tail_len + t, p.inv_freq[i], &c64, &s64);
+            const float a = __bfloat162float(src[i]), bb = __bfloat162float(src[i + D / 2]);
+            const float c32 = static_cast<float>(c64), s32 = static_cast<float>(s64);
+            y0 = rope_rotate_bf16(a, bb, c32, s32, c64, s64, true);
+            y1 = rope_rotate_bf16(a, bb, c32, s32, c64, s64, false);
+          }
+          qs[rho * D + i] = static_cast<uint16_t>(y0);
+          qs[rho * D + i + D / 2] = static_cast<uint16_t>(y1);
+        }
+        consumer_sync();
 #pragma unroll
         for (int kk = 0; kk < kKSteps; ++kk) {
           const int c0 = 16 * kk + 2 * t4;
-          qf[kk][0] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + c0) : 0u;
-          qf[kk][1] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + c0) : 0u;
-          qf[kk][2] = q0 ? *reinterpret_cast<const uint32_t*>(q0 + c0 + 8) : 0u;
-          qf[kk][3] = q1 ? *reinterpret_cast<const uint32_t*>(q1 + c0 + 8) : 0u;
+          qf[kk][0] = *reinterpret_cast<const uint32_t*>(qs + r0 * D + c0);
+          qf[kk][1] = *reinterpret_cast<const uint32_t*>(qs + r1 * D + c0);
+          qf[kk][2] = *reinterpret_cast<const uint32_t*>(qs + r0 * D + c0 + 8);
+          qf[kk][3] = *reinterpret_cast<const uint32_t*>(qs + r1 * D + c0 + 8);
         }
+        consumer_sync();  // the buffer is reused by the combine below
         q_bh = bh;
       }
       float o[D / 8][4];
@@ -388,6 +442,26 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
         if (!mbar_wait(&full[st], (gt / kDecStages) & 1, &abort_flag, p.status)) break;
         const uint32_t kb = smem_u32(sK + st * kTileBytes);
         const uint32_t vb = smem_u32(sV + st * kTileBytes);
+        // A tile that runs past the unit's last key holds rows of other units
+        // (or of this call's new tokens, which another CTA may be writing):
+        // masked keys get P = 0, but 0 * NaN would still poison P V, so each
+        // warp clears its own V rows past the end. The fence orders these
+        // generic writes before the next TMA write into the stage.
+        {
+          const int first_bad = cr.k_hi - (cr.k_lo + it * kDecTile);
+          if (first_bad < kDecTile && 16 * warp + 15 >= first_bad) {
+            uint8_t* vt = sV + st * kTileBytes;
+            for (int idx = lane; idx < 16 * (D / 64) * 8; idx += 32) {
+              const int rr = 16 * warp + idx / ((D / 64) * 8);
+              const int rem = idx % ((D / 64) * 8);
+              if (rr >= first_bad)
+                *reinterpret_cast<uint4*>(vt + (rem / 8) * kHalfBytes + rr * 128 + (rem % 8) * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+            }
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+          }
+        }
         // S = Q K^T for this warp's 16 keys (two n-tiles of 8 keys)
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         {

@@ -7,19 +7,12 @@
 // 2607.20457, "What carries the argument"]. Pair (x_i, x_{i+D/2}) turns by
 // p * theta^(-2i/D).
 //
-// Precision: the angle p * theta_i, its reduction modulo 2*pi (Cody-Waite,
-// two constants) and sine/cosine are fp64. Every output is the correctly
-// rounded bf16 (nearest even) of the exact rotation. The rotation first runs
-// in fp32 with a bound E on its error; when y - E and y + E round to the same
-// bf16 value that value is the correct rounding (Ziv's rounding test), and
-// otherwise (about one element in 10^4) the element is recomputed in fp64 and
-// rounded once through fp32 round-to-odd (Boldo and Melquiond, 2008: odd
-// rounding to a format >= 2 bits wider, then nearest, equals direct nearest
-// rounding). At p ~ 1e6 an fp32 angle would err by ~0.06 rad, and even an
-// fp32 rotation with an exact angle lands one bf16 ulp off the correct value
-// for a few elements in 1e5, enough to move a peaked softmax's log-sum-exp by
-// ~3e-2; correct rounding makes the cache reproducible bit for bit.
-// theta_i = theta^(-2i/D) comes from the host in fp64.
+// Precision: see rope_math.cuh (fp64 angles and sine/cosine; every output
+// is the correctly rounded bf16 of the exact rotation). At p ~ 1e6 an fp32
+// angle would err by ~0.06 rad, and even an fp32 rotation with an exact
+// angle lands one bf16 ulp off the correct value for a few elements in 1e5,
+// enough to move a peaked softmax's log-sum-exp by ~3e-2; correct rounding
+// makes the cache reproducible bit for bit.
 //
 // One launch handles up to three jobs (Q, K, V of one call): blockIdx.z
 // selects the job. Each CTA covers kTokPerCta tokens of one job; it first
@@ -28,24 +21,15 @@
 // chunk c of the second half of one head.
 #include <cmath>
 
+#include "rope_math.cuh"
 #include "star_common.cuh"
 #include "star_kernels.cuh"
 
 namespace star {
 
 namespace {
-// fp64 -> fp32 with round-to-odd: truncate, then force the last bit to 1 if
-// anything was cut off.
-__device__ __forceinline__ float f32_round_odd(double x) {
-  float f = __double2float_rz(x);
-  if (static_cast<double>(f) != x) f = __uint_as_float(__float_as_uint(f) | 1u);
-  return f;
-}
 constexpr int kRopeThreads = 256;
 constexpr int kTokPerCta = 8;
-constexpr double kTwoPiHi = 6.283185307179586;         // nearest double to 2*pi
-constexpr double kTwoPiLo = 2.4492935982947064e-16;    // 2*pi - kTwoPiHi
-constexpr double kInvTwoPi = 0.15915494309189535;
 }  // namespace
 
 __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constant__ RopeParams p) {
@@ -65,12 +49,8 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
       int t = e / half, i = e % half;
       int s = tok0 + t;
       long long pos = p.pos ? static_cast<long long>(p.pos[s]) : p.pos0 + s;
-      double ang = static_cast<double>(pos) * p.inv_freq[i];
-      double k = rint(ang * kInvTwoPi);
-      double r = fma(-k, kTwoPiHi, ang);
-      r = fma(-k, kTwoPiLo, r);
       double sn, cs;
-      sincos(r, &sn, &cs);
+      rope_angle(pos, p.inv_freq[i], &cs, &sn);
       s_cos[t][i] = cs;
       s_sin[t][i] = sn;
       f_cos[t][i] = static_cast<float>(cs);
@@ -98,31 +78,14 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
         const int i0 = 8 * c + 2 * w;
         const float a0 = bf16_lo(pl[w]), a1 = bf16_hi(pl[w]);
         const float b0 = bf16_lo(ph[w]), b1 = bf16_hi(ph[w]);
-        const float c0 = f_cos[t][i0], c1 = f_cos[t][i0 + 1];
-        const float s0 = f_sin[t][i0], s1 = f_sin[t][i0 + 1];
-        // |fp32 result - exact| <= 2^-22 (|a| + |b|): one rounding each for
-        // cos/sin (2^-25 relative), the product and the fused multiply-add
-        const float e0 = 2.3841858e-07f * (fabsf(a0) + fabsf(b0));
-        const float e1 = 2.3841858e-07f * (fabsf(a1) + fabsf(b1));
-        float y[4] = {fmaf(a0, c0, -(b0 * s0)), fmaf(a1, c1, -(b1 * s1)),
-                      fmaf(b0, c0, a0 * s0), fmaf(b1, c1, a1 * s1)};
-        const float err[4] = {e0, e1, e0, e1};
-        uint32_t out[4];
-#pragma unroll
-        for (int m = 0; m < 4; ++m) {
-          const uint32_t lohi = pack_bf16x2(y[m] - err[m], y[m] + err[m]);
-          if ((lohi & 0xFFFFu) == (lohi >> 16)) {
-            out[m] = lohi & 0xFFFFu;
-          } else {  // within E of a rounding boundary: decide in fp64
-            const int ii = i0 + (m & 1);
-            const double ad = (m & 1) ? a1 : a0, bd = (m & 1) ? b1 : b0;
-            const double cd = s_cos[t][ii], sd = s_sin[t][ii];
-            const double yd = (m < 2) ? ad * cd - bd * sd : bd * cd + ad * sd;
-            out[m] = pack_bf16x2(f32_round_odd(yd), 0.f) & 0xFFFFu;
-          }
-        }
-        ol[w] = out[0] | (out[1] << 16);
-        oh[w] = out[2] | (out[3] << 16);
+        ol[w] = rope_rotate_bf16(a0, b0, f_cos[t][i0], f_sin[t][i0], s_cos[t][i0], s_sin[t][i0], true) |
+                (rope_rotate_bf16(a1, b1, f_cos[t][i0 + 1], f_sin[t][i0 + 1], s_cos[t][i0 + 1],
+                                  s_sin[t][i0 + 1], true)
+                 << 16);
+        oh[w] = rope_rotate_bf16(a0, b0, f_cos[t][i0], f_sin[t][i0], s_cos[t][i0], s_sin[t][i0], false) |
+                (rope_rotate_bf16(a1, b1, f_cos[t][i0 + 1], f_sin[t][i0 + 1], s_cos[t][i0 + 1],
+                                  s_sin[t][i0 + 1], false)
+                 << 16);
       }
       lo = make_uint4(ol[0], ol[1], ol[2], ol[3]);
       hi = make_uint4(oh[0], oh[1], oh[2], oh[3]);
@@ -132,9 +95,9 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
   }
 }
 
-void rope_set_freq(RopeParams& p, int D, double theta) {
+void rope_fill_freq(double* out, int D, double theta) {
   for (int i = 0; i < 64; ++i)
-    p.inv_freq[i] = (i < D / 2) ? std::pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(D)) : 0.0;
+    out[i] = (i < D / 2) ? std::pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(D)) : 0.0;
 }
 
 cudaError_t launch_rope(const RopeParams& p, int njobs, cudaStream_t stream) {

@@ -27,8 +27,9 @@ struct RopeParams {
   long long pos0;
   double inv_freq[64];  // theta^(-2i/D), i < D/2 (fp64, from the host)
 };
-// Fills p.inv_freq for head dim D and base theta.
-void rope_set_freq(RopeParams& p, int D, double theta);
+// Fills out[0..63] with theta^(-2i/D) for i < D/2 (zero beyond).
+void rope_fill_freq(double* out, int D, double theta);
+inline void rope_set_freq(RopeParams& p, int D, double theta) { rope_fill_freq(p.inv_freq, D, theta); }
 cudaError_t launch_rope(const RopeParams& p, int njobs, cudaStream_t stream);
 
 // ---- tcgen05 attention (Phase 1, and Phase 2 query chunks) -----------------
@@ -59,7 +60,13 @@ constexpr int kMaxChunksPerSplit = 64;  // chunk size is chosen so a split has a
 struct DecodeParams {
   CUtensorMap tmK;  // K cache: dims {D, Lvalid, B*Hkv}, box {64, 64, 1}
   CUtensorMap tmV;
-  const __nv_bfloat16* q;  // rotated q [B, T, Hq, D]
+  const __nv_bfloat16* q_new;  // pre-RoPE q of the new tokens [B, T, Hq, D]
+  const __nv_bfloat16* k_new;  // pre-RoPE k [B, T, Hkv, D], appended to the cache in-kernel
+  const __nv_bfloat16* v_new;  // v [B, T, Hkv, D]
+  __nv_bfloat16* k_cache;      // [B*Hkv, Lcap, D]
+  __nv_bfloat16* v_cache;
+  int Lcap;
+  double inv_freq[64];         // theta^(-2i/D), i < D/2
   int B, T, Hq, Hkv, g, R;  // R = T * g rows (<= kDecRows)
   int L, b, n, tail_len;    // context, block length, context splits, earlier tail tokens
   int chunk;                // keys per CTA (multiple of kDecTile)

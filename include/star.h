@@ -178,7 +178,7 @@ star_status star_lse_merge(const float* part_o, const float* part_lse, int nspli
  * counterpart: this entry point exists for callers that cannot allocate
  * device memory themselves, such as a plugin whose host application owns
  * every device allocation, or a serving loop that must never block in
- * cudaMalloc/cudaFree. Its scratch (the rotated query and the per-chunk
+ * cudaMalloc/cudaFree. Its scratch (the split counters and the per-chunk
  * partials) lives in a 16 MiB device array inside the library, which every
  * GPU that loads the library keeps until the process exits; the caller still
  * passes inputs and outputs, with the same meaning and layout as
