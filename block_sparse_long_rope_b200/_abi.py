@@ -33,6 +33,7 @@ EXPORTS = (
     "star_lse_merge",
     "star_device_status",
     "star_debug_index",
+    "star_debug_wait_probe",
 )
 
 
@@ -92,6 +93,8 @@ def load(path: str = LIB_PATH):
         lib.star_lse_merge.argtypes = [_P, _P, _I, _P, _P, _I, _I, _I, _I, _P]
         lib.star_device_status.restype = _I
         lib.star_device_status.argtypes = [_P, _P]
+        lib.star_debug_wait_probe.restype = _I
+        lib.star_debug_wait_probe.argtypes = [_P, _D, _P]
         lib.star_debug_index.restype = _I
         lib.star_debug_index.argtypes = [_I, _I, _I, _P, _P, _P, _P]
         _lib = lib

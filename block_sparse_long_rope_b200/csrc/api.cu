@@ -564,6 +564,21 @@ star_status star_device_status(void* workspace, void* cuda_stream) {
   return ok();
 }
 
+star_status star_debug_wait_probe(void* workspace, double seconds, void* cuda_stream) {
+  star_status s;
+  if ((s = check_ptr(workspace, "workspace")) != STAR_OK) return s;
+  if (!(seconds > 0.0) || seconds > 2.0)
+    return fail(STAR_ERR_INVALID_ARG, "seconds must lie in (0, 2]");
+  if ((s = check_device(nullptr)) != STAR_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e = cudaMemsetAsync(workspace, 0, star::kStatusBytes, st);
+  if (e != cudaSuccess) return cuda_fail(e, "status reset");
+  e = star::launch_debug_wait_probe(static_cast<int*>(workspace),
+                                    static_cast<unsigned long long>(seconds * 1e9), st);
+  if (e != cudaSuccess) return cuda_fail(e, "wait probe launch");
+  return ok();
+}
+
 star_status star_debug_index(int L, int block_len, int anchor_len, int32_t* blk, int32_t* pos,
                              int32_t* kv_ranges, void* cuda_stream) {
   if (L < 1 || block_len < 1 || anchor_len < 0 || anchor_len > block_len)

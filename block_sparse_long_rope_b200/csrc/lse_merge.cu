@@ -112,6 +112,27 @@ __global__ void debug_index_kernel(int L, int b, int a, int32_t* blk, int32_t* p
   for (int j = 0; j < 4; ++j) ranges[4 * r + j] = out[j];
 }
 
+// One CTA waits, through the same bounded wait the attention and decode
+// kernels use, on an mbarrier that nothing arrives on: after limit_ns the
+// wait gives up and records the time-out in *status; the kernel returns.
+__global__ void debug_wait_probe_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ volatile int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    abort_flag = 0;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_flag, status, limit_ns);
+  __syncthreads();
+}
+
+cudaError_t launch_debug_wait_probe(int* status, unsigned long long limit_ns, cudaStream_t stream) {
+  debug_wait_probe_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_debug_index(int L, int b, int a, int32_t* blk, int32_t* pos, int32_t* ranges,
                                cudaStream_t stream) {
   if (L <= 0) return cudaSuccess;

@@ -96,5 +96,6 @@ void set_last_error(const char* msg);
 // ---- debug: device-evaluated index math --------------------------------------
 cudaError_t launch_debug_index(int L, int b, int a, int32_t* blk, int32_t* pos, int32_t* ranges,
                                cudaStream_t stream);
+cudaError_t launch_debug_wait_probe(int* status, unsigned long long limit_ns, cudaStream_t stream);
 
 }  // namespace star

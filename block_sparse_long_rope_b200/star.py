@@ -159,6 +159,13 @@ def star_device_status(workspace, stream=None):
     _abi.check(lib.star_device_status(_ptr(workspace), _stream(stream)))
 
 
+def star_debug_wait_probe(workspace, seconds=0.05, stream=None):
+    """Make a kernel's bounded wait run out on purpose (no fault): the
+    following star_device_status raises STAR_ERR_DEVICE_TIMEOUT."""
+    lib = _abi.load()
+    _abi.check(lib.star_debug_wait_probe(_ptr(workspace), float(seconds), _stream(stream)))
+
+
 def star_debug_index(L, block_len, anchor_len, device="cuda", stream=None):
     """Device-evaluated index math: (blk[L], pos[L], kv_ranges[L,4]) int32."""
     blk = torch.empty(L, dtype=torch.int32, device=device)

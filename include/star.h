@@ -210,6 +210,17 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
 star_status star_device_status(void* workspace, void* cuda_stream);
 
 /*
+ * star_debug_wait_probe — checks the kernels' bounded waits and the status
+ * read-back: one CTA waits, through the same bounded wait the attention and
+ * decode kernels use, on a barrier nothing arrives on; after `seconds`
+ * (0 < seconds <= 2) the wait gives up and records a time-out in the status
+ * word at the start of `workspace` (>= 256 bytes, cleared first). A following
+ * star_device_status returns STAR_ERR_DEVICE_TIMEOUT; nothing faults and the
+ * context stays usable.
+ */
+star_status star_debug_wait_probe(void* workspace, double seconds, void* cuda_stream);
+
+/*
  * star_debug_index — evaluates the kernels' index math on the device for
  * every context row r in [0, L): blk[r] = block id, pos[r] = position ID,
  * kv_ranges[4r..4r+3] = {anchor_lo, anchor_hi, own_lo, own_hi} (half-open;

@@ -144,3 +144,9 @@ def test_python_binding_raises_on_missing_library(tmp_path):
             _abi.load(str(tmp_path / "nope.so"))
     finally:
         _abi._lib = saved
+
+
+def test_wait_probe_validation(lib):
+    assert lib.star_debug_wait_probe(NULL, 0.05, NULL) == INVALID
+    assert lib.star_debug_wait_probe(FAKE, 0.0, NULL) == INVALID
+    assert lib.star_debug_wait_probe(FAKE, 3.0, NULL) == INVALID

@@ -91,3 +91,24 @@ def test_lse_merge_kernel(D):
     got_o = to64(o).transpose(0, 2, 1, 3).reshape(R, D)
     assert max_abs(got_o, ro) <= TOL_O
     assert max_abs(to64(lse).reshape(R), rl) <= TOL_LSE
+
+
+# ----------------------------------------------------------------------------- bounded waits
+def test_bounded_wait_reports_timeout_and_context_survives():
+    """A wait on a barrier nothing arrives on gives up after its limit and
+    the host reads STAR_ERR_DEVICE_TIMEOUT; afterwards the context still runs
+    kernels (a RoPE call checks out) and the status word reads clean."""
+    from block_sparse_long_rope_b200 import _abi
+
+    ws = star.alloc_workspace(256)
+    star.star_debug_wait_probe(ws, seconds=0.05)
+    with pytest.raises(_abi.StarError) as ei:
+        star.star_device_status(ws)
+    assert ei.value.name == "STAR_ERR_DEVICE_TIMEOUT"
+    star.star_device_status(ws)  # read-back cleared the word
+    x = rand_bf16((1, 4, 2, 64), seed=3)
+    y = torch.empty_like(x)
+    star.star_rope(x, y, 1e4)
+    torch.cuda.synchronize()
+    ref = orc.rope(x.cpu(), np.arange(4), 1e4, round_out=True)
+    np.testing.assert_array_equal(to64(y), ref)
