@@ -113,3 +113,49 @@ def round_bf16_np(x):
     x = np.asarray(x, dtype=np.float64)
     m, e = np.frexp(x)  # x = m * 2^e, |m| in [0.5, 1)
     return np.ldexp(np.round(m * 256.0) / 256.0, e)
+
+
+def prefix_mask(L, b, prefix):
+    """Dense mask of the generalised Phase 1 over context keys: block i >= 1
+    sees its prefix ranges prefix[i] (list of [s, e)) and, causally, itself."""
+    M = np.zeros((L, L), dtype=bool)
+    for r in range(L):
+        i = r // b
+        if i > 0:
+            for s, e in prefix[i]:
+                if e > s:
+                    M[r, s:e] = True
+        M[r, i * b:r + 1] = True
+    return M
+
+
+def explicit_anchor_literal(q, k, v, b, ak, av, apos, theta):
+    """Augmented block [explicit anchor || c_i] built literally: the anchor
+    rows (given content at given positions) then block i at its own
+    positions, rotated, plain causal attention, keep the c_i rows.
+    q[L,Hq,D], k/v[L,Hkv,D], ak/av[La,Hkv,D] pre-RoPE float64."""
+    L, Hq, D = q.shape
+    Hkv = k.shape[1]
+    g = Hq // Hkv
+    La = ak.shape[0]
+    o = np.empty_like(q)
+    lse = np.empty((Hq, L))
+    for i in range(-(-L // b)):
+        own = np.arange(i * b, min((i + 1) * b, L))
+        qo = rope_complex(q[own], own, theta)
+        ko = rope_complex(k[own], own, theta)
+        if i > 0:
+            kk = np.concatenate([rope_complex(ak, np.asarray(apos), theta), ko], axis=0)
+            vv = np.concatenate([av, v[own]], axis=0)
+        else:
+            kk, vv = ko, v[own]
+        na = kk.shape[0] - own.size
+        # row j of the block sees the whole anchor and block rows 0..j
+        mask = np.zeros((own.size, kk.shape[0]), dtype=bool)
+        mask[:, :na] = True
+        mask[:, na:] = np.tril(np.ones((own.size, own.size), dtype=bool))
+        for h in range(Hq):
+            oo, ll = masked_attention(qo[:, h], kk[:, h // g], vv[:, h // g], mask)
+            o[own, h] = oo
+            lse[h, own] = ll
+    return o, lse

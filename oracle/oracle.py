@@ -33,6 +33,9 @@ def _load():
             lib.orc_phase1_rows_sel.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I,
                                                 ctypes.c_double, ctypes.c_int, _I, _P, _P, _P,
                                                 _P, _P, _P]
+            lib.orc_phase1_ext_rows.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P,
+                                                _P, _I, ctypes.c_double, ctypes.c_int, _I, _P,
+                                                _P, _P, _P, _P, _P]
             lib.orc_phase2_rows.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                             _I, _I, ctypes.c_double, ctypes.c_int, _I, _P,
                                             _P, _P, _P, _P]
@@ -41,7 +44,7 @@ def _load():
                                             _P, _P, _P]
             lib.orc_lse_merge.argtypes = [_P, _P, _I, _I, _I, _P, _P]
             for f in ("orc_round_bf16", "orc_rope", "orc_phase1_ranges", "orc_phase1_rows",
-                      "orc_phase1_rows_sel",
+                      "orc_phase1_rows_sel", "orc_phase1_ext_rows",
                       "orc_phase2_rows", "orc_global_rows", "orc_lse_merge"):
                 getattr(lib, f).restype = None
             _lib = lib
@@ -124,6 +127,42 @@ def phase1_rows_selected(q_sel, k, v, block_len, anchor_len, theta, qb, qh, qr, 
     _load().orc_phase1_rows_sel(_ptr(qbits), _ptr(kbits), _ptr(vbits), L, Hq, Hkv, D, block_len,
                                 anchor_len, float(theta), int(bool(round_qk)), nq, _ptr(qb),
                                 _ptr(qh), _ptr(qr), _ptr(o), _ptr(lse), _ptr(nvis))
+    return o, lse, nvis
+
+
+def phase1_ext_rows(q, k, v, block_len, prefix, theta, qb, qh, qr, anchor_k=None, anchor_v=None,
+                    anchor_pos=None, round_qk=True):
+    """Generalised Phase 1 for the listed queries: prefix[n, R, 2] int ranges
+    [s, e) of context rows per block (e <= s unused), plus an optional explicit
+    anchor (anchor_k/v [B, La, Hkv, D] bf16 rotated at anchor_pos[La])."""
+    qbits, kbits, vbits = bf16_bits(q), bf16_bits(k), bf16_bits(v)
+    B, L, Hq, D = qbits.shape
+    Hkv = kbits.shape[2]
+    pre = np.ascontiguousarray(np.asarray(prefix, dtype=np.int64))
+    n = -(-L // block_len)
+    assert pre.ndim == 3 and pre.shape[0] == n and pre.shape[2] == 2
+    R = pre.shape[1]
+    if anchor_k is None:
+        ak = np.zeros((1,), dtype=np.uint16)
+        av = ak
+        ap = np.zeros((1,), dtype=np.int64)
+        La = 0
+    else:
+        ak, av = bf16_bits(anchor_k), bf16_bits(anchor_v)
+        La = ak.shape[1]
+        ap = np.ascontiguousarray(np.asarray(anchor_pos, dtype=np.int64))
+        assert ap.shape == (La,)
+    qb = np.ascontiguousarray(qb, dtype=np.int64)
+    qh = np.ascontiguousarray(qh, dtype=np.int64)
+    qr = np.ascontiguousarray(qr, dtype=np.int64)
+    nq = qb.size
+    o = np.empty((nq, D), dtype=np.float64)
+    lse = np.empty((nq,), dtype=np.float64)
+    nvis = np.empty((nq,), dtype=np.int64)
+    _load().orc_phase1_ext_rows(_ptr(qbits), _ptr(kbits), _ptr(vbits), L, Hq, Hkv, D, block_len,
+                                _ptr(pre), R, _ptr(ak), _ptr(av), _ptr(ap), La, float(theta),
+                                int(bool(round_qk)), nq, _ptr(qb), _ptr(qh), _ptr(qr), _ptr(o),
+                                _ptr(lse), _ptr(nvis))
     return o, lse, nvis
 
 

@@ -270,6 +270,73 @@ void orc_phase1_rows_sel(const uint16_t* q_sel_bits, const uint16_t* k_bits,
                    round_qk, nq, qb, qh, qr, o, lse, nvis);
 }
 
+// Generalised Phase 1 (prefix variants). Row r of block i = r / b sees
+//   i == 0 : [0, r]                                    (c'_1 = c_1, causal)
+//   i >= 1 : the explicit anchor keys (all La, if given)
+//            U the block's prefix ranges of context rows [s, e), e <= i*b,
+//              at their original positions
+//            U [i*b, r] (own block, causal)
+// The Star anchor is the prefix {[0, a)}; no anchor is the empty prefix
+// (pith 2WVXFXZ2 "What carries the argument"; the anchor ablations in the
+// atlas.scime.ai measured-effects table: no anchor, anchor position IDs
+// changed, anchor content replaced); Pulsar's layout is a 64-token sink plus
+// chunks of earlier blocks at their original positions (pith 2607.20457,
+// "What carries the argument"). The explicit anchor (ak/av[B, La, Hkv, D],
+// positions apos[La]) is rotated at apos. prefix[(i*R + j)*2 + {0,1}] =
+// {s, e}; e <= s marks an unused slot. Key index c < L is context row c,
+// c >= L is explicit anchor key c - L.
+void orc_phase1_ext_rows(const uint16_t* q_bits, const uint16_t* k_bits, const uint16_t* v_bits,
+                         i64 L, i64 Hq, i64 Hkv, i64 D, i64 block_len, const i64* prefix, i64 R,
+                         const uint16_t* ak_bits, const uint16_t* av_bits, const i64* apos, i64 La,
+                         double theta, int round_qk, i64 nq, const i64* qb, const i64* qh,
+                         const i64* qr, double* o, double* lse, i64* nvis) {
+  const i64 g = Hq / Hkv;
+  const double scale = 1.0 / std::sqrt(static_cast<double>(D));
+  std::map<std::pair<i64, i64>, std::vector<i64>> groups;
+  for (i64 i = 0; i < nq; ++i) groups[{qb[i], qh[i] / g}].push_back(i);
+  for (auto& kv : groups) {
+    const i64 b = kv.first.first, kvh = kv.first.second;
+    i64 nmax = 0;
+    for (i64 i : kv.second) nmax = std::max(nmax, qr[i] + 1);
+    std::vector<double> K = rope_rows(k_bits, b, kvh, nmax, L, Hkv, D, 0, theta, round_qk != 0);
+    std::vector<double> V = plain_rows(v_bits, b, kvh, nmax, L, Hkv, D);
+    std::vector<double> AK(static_cast<size_t>(La * D)), AV(static_cast<size_t>(La * D));
+    for (i64 c = 0; c < La; ++c) {
+      std::vector<double> x(D);
+      const uint16_t* src = ak_bits + ((b * La + c) * Hkv + kvh) * D;
+      for (i64 d = 0; d < D; ++d) x[d] = bf16_to_double(src[d]);
+      rope_vec(x.data(), AK.data() + c * D, D, static_cast<double>(apos[c]), theta);
+      if (round_qk)
+        for (i64 d = 0; d < D; ++d) AK[c * D + d] = round_to_bf16(AK[c * D + d]);
+      const uint16_t* vs = av_bits + ((b * La + c) * Hkv + kvh) * D;
+      for (i64 d = 0; d < D; ++d) AV[c * D + d] = bf16_to_double(vs[d]);
+    }
+    auto key = [&](i64 c) { return c < L ? K.data() + c * D : AK.data() + (c - L) * D; };
+    auto val = [&](i64 c) { return c < L ? V.data() + c * D : AV.data() + (c - L) * D; };
+    const std::vector<i64>& qs = kv.second;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (size_t j = 0; j < qs.size(); ++j) {
+      const i64 i = qs[j], r = qr[i], blk = r / block_len;
+      std::vector<double> x(D), q(D);
+      const uint16_t* src = q_bits + ((b * L + r) * Hq + qh[i]) * D;
+      for (i64 d = 0; d < D; ++d) x[d] = bf16_to_double(src[d]);
+      rope_vec(x.data(), q.data(), D, static_cast<double>(r), theta);
+      if (round_qk)
+        for (i64 d = 0; d < D; ++d) q[d] = round_to_bf16(q[d]);
+      std::vector<Range> vis;
+      if (blk > 0) {
+        if (La > 0) vis.push_back({L, L + La});
+        for (i64 t = 0; t < R; ++t) {
+          const i64 s0 = prefix[(blk * R + t) * 2], e0 = prefix[(blk * R + t) * 2 + 1];
+          if (e0 > s0) vis.push_back({s0, e0});
+        }
+      }
+      vis.push_back({blk * block_len, r + 1});
+      attend(q.data(), D, scale, vis, key, val, o + i * D, lse + i, nvis ? nvis + i : nullptr);
+    }
+  }
+}
+
 // Phase 2 partials ([pith 2WVXFXZ2, Referee summary and Circularity check]):
 // for new token t of this call (query or decode; position L + tail_len + t),
 // one (normalised output, LSE) pair per split:
