@@ -7,7 +7,7 @@ from .oracle import (  # noqa: F401
     bf16_bits,
     global_rows,
     lse_merge,
-    phase1_ext_rows,
+    phase1_gather_rows,
     phase1_full,
     phase1_ranges,
     phase1_rows,

@@ -116,41 +116,43 @@ def round_bf16_np(x):
 
 
 def prefix_mask(L, b, prefix):
-    """Dense mask of the generalised Phase 1 over context keys: block i >= 1
-    sees its prefix ranges prefix[i] (list of [s, e)) and, causally, itself."""
+    """Dense mask of the generalised Phase 1 over context keys: block i sees
+    the context rows of its ranges prefix[i] (list of [s, e)) and, causally,
+    itself."""
     M = np.zeros((L, L), dtype=bool)
     for r in range(L):
         i = r // b
-        if i > 0:
-            for s, e in prefix[i]:
-                if e > s:
-                    M[r, s:e] = True
+        for s, e in prefix[i]:
+            if e > s:
+                M[r, s:e] = True
         M[r, i * b:r + 1] = True
     return M
 
 
-def explicit_anchor_literal(q, k, v, b, ak, av, apos, theta):
-    """Augmented block [explicit anchor || c_i] built literally: the anchor
-    rows (given content at given positions) then block i at its own
-    positions, rotated, plain causal attention, keep the c_i rows.
-    q[L,Hq,D], k/v[L,Hkv,D], ak/av[La,Hkv,D] pre-RoPE float64."""
+def gathered_prefix_literal(q, k, v, b, pk, pv, ppos, bounds, theta):
+    """Augmented block [prefix rows || c_i] built literally: block i takes
+    the prefix rows pk/pv[bounds[i,0]:bounds[i,1]] (pre-RoPE content, keys
+    rotated at ppos), then itself at its own positions; plain causal
+    attention in which every prefix row is visible; keep the c_i rows.
+    q[L,Hq,D], k/v[L,Hkv,D], pk/pv[G,Hkv,D] float64, ppos[G]."""
     L, Hq, D = q.shape
     Hkv = k.shape[1]
     g = Hq // Hkv
-    La = ak.shape[0]
     o = np.empty_like(q)
     lse = np.empty((Hq, L))
+    ppos = np.asarray(ppos)
     for i in range(-(-L // b)):
         own = np.arange(i * b, min((i + 1) * b, L))
         qo = rope_complex(q[own], own, theta)
         ko = rope_complex(k[own], own, theta)
-        if i > 0:
-            kk = np.concatenate([rope_complex(ak, np.asarray(apos), theta), ko], axis=0)
-            vv = np.concatenate([av, v[own]], axis=0)
+        gs, ge = bounds[i]
+        if ge > gs:
+            kk = np.concatenate([rope_complex(pk[gs:ge], ppos[gs:ge], theta), ko], axis=0)
+            vv = np.concatenate([pv[gs:ge], v[own]], axis=0)
         else:
             kk, vv = ko, v[own]
         na = kk.shape[0] - own.size
-        # row j of the block sees the whole anchor and block rows 0..j
+        # row j of the block sees every prefix row and block rows 0..j
         mask = np.zeros((own.size, kk.shape[0]), dtype=bool)
         mask[:, :na] = True
         mask[:, na:] = np.tril(np.ones((own.size, own.size), dtype=bool))

@@ -33,9 +33,9 @@ def _load():
             lib.orc_phase1_rows_sel.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I,
                                                 ctypes.c_double, ctypes.c_int, _I, _P, _P, _P,
                                                 _P, _P, _P]
-            lib.orc_phase1_ext_rows.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _P, _I, _P, _P,
-                                                _P, _I, ctypes.c_double, ctypes.c_int, _I, _P,
-                                                _P, _P, _P, _P, _P]
+            lib.orc_phase1_gather_rows.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _I,
+                                                   _P, _P, _P, _I, ctypes.c_double, ctypes.c_int,
+                                                   _I, _P, _P, _P, _P, _P, _P]
             lib.orc_phase2_rows.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                             _I, _I, ctypes.c_double, ctypes.c_int, _I, _P,
                                             _P, _P, _P, _P]
@@ -44,7 +44,7 @@ def _load():
                                             _P, _P, _P]
             lib.orc_lse_merge.argtypes = [_P, _P, _I, _I, _I, _P, _P]
             for f in ("orc_round_bf16", "orc_rope", "orc_phase1_ranges", "orc_phase1_rows",
-                      "orc_phase1_rows_sel", "orc_phase1_ext_rows",
+                      "orc_phase1_rows_sel", "orc_phase1_gather_rows",
                       "orc_phase2_rows", "orc_global_rows", "orc_lse_merge"):
                 getattr(lib, f).restype = None
             _lib = lib
@@ -130,28 +130,31 @@ def phase1_rows_selected(q_sel, k, v, block_len, anchor_len, theta, qb, qh, qr, 
     return o, lse, nvis
 
 
-def phase1_ext_rows(q, k, v, block_len, prefix, theta, qb, qh, qr, anchor_k=None, anchor_v=None,
-                    anchor_pos=None, round_qk=True):
-    """Generalised Phase 1 for the listed queries: prefix[n, R, 2] int ranges
-    [s, e) of context rows per block (e <= s unused), plus an optional explicit
-    anchor (anchor_k/v [B, La, Hkv, D] bf16 rotated at anchor_pos[La])."""
+def phase1_gather_rows(q, k, v, block_len, src, pos, bounds, theta, qb, qh, qr, extra_k=None,
+                       extra_v=None, round_qk=True):
+    """Generalised Phase 1 for the listed queries. The prefix table has G
+    rows: row t is context row src[t] (src >= 0) or extra row -1 - src[t]
+    (extra_k/v [B, NX, Hkv, D] bf16), its key rotated at pos[t]; block i sees
+    table rows [bounds[i, 0], bounds[i, 1]) and, causally, itself."""
     qbits, kbits, vbits = bf16_bits(q), bf16_bits(k), bf16_bits(v)
     B, L, Hq, D = qbits.shape
     Hkv = kbits.shape[2]
-    pre = np.ascontiguousarray(np.asarray(prefix, dtype=np.int64))
     n = -(-L // block_len)
-    assert pre.ndim == 3 and pre.shape[0] == n and pre.shape[2] == 2
-    R = pre.shape[1]
-    if anchor_k is None:
-        ak = np.zeros((1,), dtype=np.uint16)
-        av = ak
-        ap = np.zeros((1,), dtype=np.int64)
-        La = 0
+    src = np.ascontiguousarray(np.asarray(src, dtype=np.int64).reshape(-1))
+    pos = np.ascontiguousarray(np.asarray(pos, dtype=np.int64).reshape(-1))
+    G = src.size
+    assert pos.shape == (G,)
+    bnd = np.ascontiguousarray(np.asarray(bounds, dtype=np.int64))
+    assert bnd.shape == (n, 2)
+    assert ((0 <= bnd) & (bnd <= G)).all()
+    if extra_k is None:
+        xk = np.zeros((1,), dtype=np.uint16)
+        xv = xk
+        NX = 0
     else:
-        ak, av = bf16_bits(anchor_k), bf16_bits(anchor_v)
-        La = ak.shape[1]
-        ap = np.ascontiguousarray(np.asarray(anchor_pos, dtype=np.int64))
-        assert ap.shape == (La,)
+        xk, xv = bf16_bits(extra_k), bf16_bits(extra_v)
+        NX = xk.shape[1]
+    assert ((src < L) & (src >= -NX)).all()
     qb = np.ascontiguousarray(qb, dtype=np.int64)
     qh = np.ascontiguousarray(qh, dtype=np.int64)
     qr = np.ascontiguousarray(qr, dtype=np.int64)
@@ -159,10 +162,10 @@ def phase1_ext_rows(q, k, v, block_len, prefix, theta, qb, qh, qr, anchor_k=None
     o = np.empty((nq, D), dtype=np.float64)
     lse = np.empty((nq,), dtype=np.float64)
     nvis = np.empty((nq,), dtype=np.int64)
-    _load().orc_phase1_ext_rows(_ptr(qbits), _ptr(kbits), _ptr(vbits), L, Hq, Hkv, D, block_len,
-                                _ptr(pre), R, _ptr(ak), _ptr(av), _ptr(ap), La, float(theta),
-                                int(bool(round_qk)), nq, _ptr(qb), _ptr(qh), _ptr(qr), _ptr(o),
-                                _ptr(lse), _ptr(nvis))
+    _load().orc_phase1_gather_rows(_ptr(qbits), _ptr(kbits), _ptr(vbits), L, Hq, Hkv, D,
+                                   block_len, _ptr(src), _ptr(pos), G, _ptr(bnd), _ptr(xk),
+                                   _ptr(xv), NX, float(theta), int(bool(round_qk)), nq, _ptr(qb),
+                                   _ptr(qh), _ptr(qr), _ptr(o), _ptr(lse), _ptr(nvis))
     return o, lse, nvis
 
 

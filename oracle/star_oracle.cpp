@@ -270,26 +270,27 @@ void orc_phase1_rows_sel(const uint16_t* q_sel_bits, const uint16_t* k_bits,
                    round_qk, nq, qb, qh, qr, o, lse, nvis);
 }
 
-// Generalised Phase 1 (prefix variants). Row r of block i = r / b sees
-//   i == 0 : [0, r]                                    (c'_1 = c_1, causal)
-//   i >= 1 : the explicit anchor keys (all La, if given)
-//            U the block's prefix ranges of context rows [s, e), e <= i*b,
-//              at their original positions
-//            U [i*b, r] (own block, causal)
-// The Star anchor is the prefix {[0, a)}; no anchor is the empty prefix
-// (pith 2WVXFXZ2 "What carries the argument"; the anchor ablations in the
-// atlas.scime.ai measured-effects table: no anchor, anchor position IDs
-// changed, anchor content replaced); Pulsar's layout is a 64-token sink plus
-// chunks of earlier blocks at their original positions (pith 2607.20457,
-// "What carries the argument"). The explicit anchor (ak/av[B, La, Hkv, D],
-// positions apos[La]) is rotated at apos. prefix[(i*R + j)*2 + {0,1}] =
-// {s, e}; e <= s marks an unused slot. Key index c < L is context row c,
-// c >= L is explicit anchor key c - L.
-void orc_phase1_ext_rows(const uint16_t* q_bits, const uint16_t* k_bits, const uint16_t* v_bits,
-                         i64 L, i64 Hq, i64 Hkv, i64 D, i64 block_len, const i64* prefix, i64 R,
-                         const uint16_t* ak_bits, const uint16_t* av_bits, const i64* apos, i64 La,
-                         double theta, int round_qk, i64 nq, const i64* qb, const i64* qh,
-                         const i64* qr, double* o, double* lse, i64* nvis) {
+// Generalised Phase 1 (gathered prefix). A prefix table of G rows: row g
+// holds the key/value of context row src[g] (src[g] >= 0) or of extra row
+// -1 - src[g] (xk/xv[B, NX, Hkv, D]), and its key is rotated at position
+// pos[g]. Row r of block i = r / b sees
+//   the prefix rows g in [bounds[2i], bounds[2i+1])   (all visible)
+//   U [i*b, r]                                        (own block, causal)
+// The Star anchor is the table of rows 0..a-1 at their own positions, seen
+// by every block i >= 1 (pith 2WVXFXZ2, "What carries the argument"); the
+// anchor ablations (atlas.scime.ai summary, measured-effects table) remove
+// it, move its position IDs or replace its content; Pulsar's layout
+// [sink || Sigma_0 || ... || Sigma_{i-1} || B_i] is the table sink, Sigma_0,
+// Sigma_1, ... with block i seeing its first 64 + |Sigma_0| + ... +
+// |Sigma_{i-1}| rows, every row at its original global position (pith
+// 2607.20457, "What carries the argument"). A row listed twice counts twice.
+// Key index c < L is context row c (own block), c >= L is prefix row c - L.
+void orc_phase1_gather_rows(const uint16_t* q_bits, const uint16_t* k_bits,
+                            const uint16_t* v_bits, i64 L, i64 Hq, i64 Hkv, i64 D, i64 block_len,
+                            const i64* src, const i64* pos, i64 G, const i64* bounds,
+                            const uint16_t* xk_bits, const uint16_t* xv_bits, i64 NX, double theta,
+                            int round_qk, i64 nq, const i64* qb, const i64* qh, const i64* qr,
+                            double* o, double* lse, i64* nvis) {
   const i64 g = Hq / Hkv;
   const double scale = 1.0 / std::sqrt(static_cast<double>(D));
   std::map<std::pair<i64, i64>, std::vector<i64>> groups;
@@ -300,37 +301,35 @@ void orc_phase1_ext_rows(const uint16_t* q_bits, const uint16_t* k_bits, const u
     for (i64 i : kv.second) nmax = std::max(nmax, qr[i] + 1);
     std::vector<double> K = rope_rows(k_bits, b, kvh, nmax, L, Hkv, D, 0, theta, round_qk != 0);
     std::vector<double> V = plain_rows(v_bits, b, kvh, nmax, L, Hkv, D);
-    std::vector<double> AK(static_cast<size_t>(La * D)), AV(static_cast<size_t>(La * D));
-    for (i64 c = 0; c < La; ++c) {
+    // the prefix table of this (batch, kv head)
+    std::vector<double> PK(static_cast<size_t>(G * D)), PV(static_cast<size_t>(G * D));
+    for (i64 t = 0; t < G; ++t) {
+      const uint16_t* ks = src[t] >= 0 ? k_bits + ((b * L + src[t]) * Hkv + kvh) * D
+                                       : xk_bits + ((b * NX + (-1 - src[t])) * Hkv + kvh) * D;
+      const uint16_t* vs = src[t] >= 0 ? v_bits + ((b * L + src[t]) * Hkv + kvh) * D
+                                       : xv_bits + ((b * NX + (-1 - src[t])) * Hkv + kvh) * D;
       std::vector<double> x(D);
-      const uint16_t* src = ak_bits + ((b * La + c) * Hkv + kvh) * D;
-      for (i64 d = 0; d < D; ++d) x[d] = bf16_to_double(src[d]);
-      rope_vec(x.data(), AK.data() + c * D, D, static_cast<double>(apos[c]), theta);
+      for (i64 d = 0; d < D; ++d) x[d] = bf16_to_double(ks[d]);
+      rope_vec(x.data(), PK.data() + t * D, D, static_cast<double>(pos[t]), theta);
       if (round_qk)
-        for (i64 d = 0; d < D; ++d) AK[c * D + d] = round_to_bf16(AK[c * D + d]);
-      const uint16_t* vs = av_bits + ((b * La + c) * Hkv + kvh) * D;
-      for (i64 d = 0; d < D; ++d) AV[c * D + d] = bf16_to_double(vs[d]);
+        for (i64 d = 0; d < D; ++d) PK[t * D + d] = round_to_bf16(PK[t * D + d]);
+      for (i64 d = 0; d < D; ++d) PV[t * D + d] = bf16_to_double(vs[d]);
     }
-    auto key = [&](i64 c) { return c < L ? K.data() + c * D : AK.data() + (c - L) * D; };
-    auto val = [&](i64 c) { return c < L ? V.data() + c * D : AV.data() + (c - L) * D; };
+    auto key = [&](i64 c) { return c < L ? K.data() + c * D : PK.data() + (c - L) * D; };
+    auto val = [&](i64 c) { return c < L ? V.data() + c * D : PV.data() + (c - L) * D; };
     const std::vector<i64>& qs = kv.second;
 #pragma omp parallel for schedule(dynamic, 1)
     for (size_t j = 0; j < qs.size(); ++j) {
       const i64 i = qs[j], r = qr[i], blk = r / block_len;
       std::vector<double> x(D), q(D);
-      const uint16_t* src = q_bits + ((b * L + r) * Hq + qh[i]) * D;
-      for (i64 d = 0; d < D; ++d) x[d] = bf16_to_double(src[d]);
+      const uint16_t* qsrc = q_bits + ((b * L + r) * Hq + qh[i]) * D;
+      for (i64 d = 0; d < D; ++d) x[d] = bf16_to_double(qsrc[d]);
       rope_vec(x.data(), q.data(), D, static_cast<double>(r), theta);
       if (round_qk)
         for (i64 d = 0; d < D; ++d) q[d] = round_to_bf16(q[d]);
       std::vector<Range> vis;
-      if (blk > 0) {
-        if (La > 0) vis.push_back({L, L + La});
-        for (i64 t = 0; t < R; ++t) {
-          const i64 s0 = prefix[(blk * R + t) * 2], e0 = prefix[(blk * R + t) * 2 + 1];
-          if (e0 > s0) vis.push_back({s0, e0});
-        }
-      }
+      const i64 gs = bounds[2 * blk], ge = bounds[2 * blk + 1];
+      if (ge > gs) vis.push_back({L + gs, L + ge});
       vis.push_back({blk * block_len, r + 1});
       attend(q.data(), D, scale, vis, key, val, o + i * D, lse + i, nvis ? nvis + i : nullptr);
     }
