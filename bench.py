@@ -308,6 +308,39 @@ def run_star(args, w, rank, world, local_rank):
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks([s2.elapsed_time(e2)], dev, world)[0]
 
+    # ---- generalised prefix: Pulsar's layout on the same workload (a side
+    # measurement outside the step: sink + 12.5% chunk summaries per block)
+    pulsar = None
+    if args.pulsar:
+        from block_sparse_long_rope_b200 import prefix as pfx
+        chunks = pfx.draw_chunks(w.L, w.block_len, seed=cfg_index)
+        src, pos, bounds = pfx.pulsar_table(w.L, w.block_len, chunks)
+        layer.set_prefix(src, pos, bounds)
+        run = lambda: layer.encode(*ctx)  # noqa: E731
+        if args.graph:
+            run()
+            torch.cuda.synchronize()
+            gp = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gp):
+                layer.encode(*ctx)
+            run = gp.replay
+        for _ in range(args.warmup):
+            run()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        s3 = torch.cuda.Event(enable_timing=True)
+        e3 = torch.cuda.Event(enable_timing=True)
+        s3.record(stream)
+        for _ in range(args.steps):
+            run()
+        e3.record(stream)
+        torch.cuda.synchronize()
+        star.star_device_status(layer.ws_phase1)
+        layer.set_prefix(None, None, None)
+        pul_ms = max_over_ranks([s3.elapsed_time(e3) / args.steps], dev, world)[0]
+        pulsar = (pul_ms, pfx.prefix_pairs(w.L, w.block_len, bounds), int(src.size))
+
     if rank != 0:
         return None
 
@@ -355,6 +388,16 @@ def run_star(args, w, rank, world, local_rank):
                        "unmasked_tflops": round(p1_tflops, 2),
                        "frac_bf16_peak": round(p1_tflops / bf16_peak, 4),
                        "note": "star_phase1_encode call: RoPE kernel + attention kernel"},
+            **({} if pulsar is None else {"phase1_pulsar_layout": {
+                "ms": round(pulsar[0], 4), "ctx_tok_s": round(w.B * w.L / (pulsar[0] / 1e3), 1),
+                "unmasked_tflops": round(4.0 * w.D * w.Hq * w.B * pulsar[1] / (pulsar[0] / 1e3) / 1e12, 2),
+                "frac_bf16_peak": round(4.0 * w.D * w.Hq * w.B * pulsar[1] / (pulsar[0] / 1e3) / 1e12 / bf16_peak, 4),
+                "table_rows": pulsar[2],
+                "speedup_vs_star_phase1": round(p1_s * 1e3 / pulsar[0], 3),
+                "note": "star_phase1_encode_ext: 64-token sink + per-block summaries of 32-token "
+                        "chunks (12.5% of a block, seeded draw standing in for Max-IDF); block i "
+                        "sees sink + summaries of blocks < i at original positions; "
+                        "gather/rope + rope + attention kernels"}}),
             "phase2_query_chunk": {"ms": round(chunk_s * 1e3, 4), "tokens": w.Tq,
                                    "tflops": round(4.0 * w.D * w.Hq * w.B * w.Tq * w.L / chunk_s / 1e12, 2)},
             "phase2_decode": {"ms": round(dec_s * 1e3, 4), "tok_s": round(dec_tok_s, 1),
@@ -427,6 +470,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", dest="cpu_baseline", action="store_false")
     ap.add_argument("--eager", dest="graph", action="store_false",
                     help="launch every call directly instead of replaying CUDA graphs")
+    ap.add_argument("--no-pulsar", dest="pulsar", action="store_false",
+                    help="skip the side measurement of Phase 1 with Pulsar's prefix layout")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=8.0)
     args = ap.parse_args()

@@ -253,17 +253,45 @@ size_t star_phase1_workspace_bytes(int B, int L, int Hq, int D) {
   return star::kStatusBytes + align_up((size_t)B * L * Hq * D * 2);
 }
 
-star_status star_phase1_encode(const void* q, const void* k, const void* v, void* o, void* k_cache,
-                               void* v_cache, int Lcap, float* lse, int B, int L, int Hq, int Hkv,
-                               int D, int block_len, int anchor_len, double theta, void* workspace,
-                               size_t workspace_bytes, void* cuda_stream) {
+size_t star_phase1_ext_workspace_bytes(int B, int L, int Hq, int Hkv, int D, int G) {
+  if (B < 1 || L < 1 || Hq < 1 || Hkv < 1 || D < 1 || G < 0) return star::kStatusBytes;
+  return star_phase1_workspace_bytes(B, L, Hq, D) + 2 * align_up((size_t)B * Hkv * G * D * 2);
+}
+
+}  // extern "C"
+
+namespace {
+
+// Body of star_phase1_encode / star_phase1_encode_ext. ext == false is the
+// Star anchor [0, anchor_len) read in place from the cache; ext == true
+// gathers the prefix table (src, pos, G rows; extra rows xk/xv) into the
+// workspace and gives block i the slice bounds[i].
+star_status phase1_run(const void* q, const void* k, const void* v, void* o, void* k_cache,
+                       void* v_cache, int Lcap, float* lse, int B, int L, int Hq, int Hkv, int D,
+                       int block_len, int anchor_len, bool ext, const int32_t* src,
+                       const int32_t* pos, int G, const int32_t* bounds, const void* xk,
+                       const void* xv, int NX, double theta, void* workspace,
+                       size_t workspace_bytes, void* cuda_stream) {
   star_status s;
   if ((s = check_heads(B, Hq, Hkv, D)) != STAR_OK) return s;
   if (L < 1) return fail(STAR_ERR_INVALID_ARG, "L must be >= 1");
   if (block_len < 1) return fail(STAR_ERR_INVALID_ARG, "block_len must be >= 1");
-  if (anchor_len < 0 || anchor_len > block_len)
+  if (!ext && (anchor_len < 0 || anchor_len > block_len))
     return fail(STAR_ERR_INVALID_ARG, "anchor_len (%d) must lie in [0, block_len=%d]", anchor_len,
                 block_len);
+  if (ext) {
+    if (G < 0) return fail(STAR_ERR_INVALID_ARG, "prefix table rows (%d) must be >= 0", G);
+    if (NX < 0) return fail(STAR_ERR_INVALID_ARG, "extra rows (%d) must be >= 0", NX);
+    if (G > 0) {
+      if (!src || (reinterpret_cast<uintptr_t>(src) & 3u))
+        return fail(STAR_ERR_INVALID_ARG, "prefix_src is NULL or not 4-byte aligned");
+      if (!pos || (reinterpret_cast<uintptr_t>(pos) & 3u))
+        return fail(STAR_ERR_INVALID_ARG, "prefix_pos is NULL or not 4-byte aligned");
+      if (!bounds || (reinterpret_cast<uintptr_t>(bounds) & 3u))
+        return fail(STAR_ERR_INVALID_ARG, "prefix_bounds is NULL or not 4-byte aligned");
+    }
+    if (NX > 0 && ((s = check_ptr(xk, "extra_k")) || (s = check_ptr(xv, "extra_v")))) return s;
+  }
   if (Lcap < L) return fail(STAR_ERR_INVALID_ARG, "Lcap (%d) < L (%d)", Lcap, L);
   if (!(theta > 0.0)) return fail(STAR_ERR_INVALID_ARG, "theta must be > 0");
   if ((s = check_ptr(q, "q")) || (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) ||
@@ -272,7 +300,8 @@ star_status star_phase1_encode(const void* q, const void* k, const void* v, void
     return s;
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
     return fail(STAR_ERR_INVALID_ARG, "lse is not 4-byte aligned");
-  const size_t need = star_phase1_workspace_bytes(B, L, Hq, D);
+  const size_t need = ext ? star_phase1_ext_workspace_bytes(B, L, Hq, Hkv, D, G)
+                          : star_phase1_workspace_bytes(B, L, Hq, D);
   if (workspace_bytes < need)
     return fail(STAR_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
   if ((long long)B * Hkv > (1ll << 31) - 1) return fail(STAR_ERR_INVALID_ARG, "B*Hkv too large");
@@ -281,6 +310,11 @@ star_status star_phase1_encode(const void* q, const void* k, const void* v, void
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   __nv_bfloat16* qrot = reinterpret_cast<__nv_bfloat16*>(ws + star::kStatusBytes);
+  const size_t qrot_bytes = align_up((size_t)B * L * Hq * D * 2);
+  const size_t tbl_bytes = align_up((size_t)B * Hkv * G * D * 2);
+  __nv_bfloat16* pk_buf = reinterpret_cast<__nv_bfloat16*>(ws + star::kStatusBytes + qrot_bytes);
+  __nv_bfloat16* pv_buf =
+      reinterpret_cast<__nv_bfloat16*>(ws + star::kStatusBytes + qrot_bytes + tbl_bytes);
   cudaError_t e = cudaMemsetAsync(ws, 0, star::kStatusBytes, st);
   if (e != cudaSuccess) return cuda_fail(e, "status reset");
 
@@ -306,12 +340,42 @@ star_status star_phase1_encode(const void* q, const void* k, const void* v, void
   star::rope_set_freq(rp, D, theta);
   e = star::launch_rope(rp, 3, st);
   if (e != cudaSuccess) return cuda_fail(e, "rope launch");
+  if (ext && G > 0) {
+    // the prefix table: K gathered and rotated at pos, V gathered, both
+    // head-major [B, Hkv, G, D] in the workspace
+    star::RopeParams rt{};
+    const long long cs[3] = {(long long)L * Hkv * D, (long long)Hkv * D, D};
+    const long long xs[3] = {(long long)NX * Hkv * D, (long long)Hkv * D, D};
+    const long long ts[3] = {(long long)Hkv * G * D, D, (long long)G * D};
+    rt.job[0] = star::RopeJob{static_cast<const __nv_bfloat16*>(k), pk_buf, {cs[0], cs[1], cs[2]},
+                              {ts[0], ts[1], ts[2]}, Hkv, 1,
+                              static_cast<const __nv_bfloat16*>(xk), {xs[0], xs[1], xs[2]}};
+    rt.job[1] = star::RopeJob{static_cast<const __nv_bfloat16*>(v), pv_buf, {cs[0], cs[1], cs[2]},
+                              {ts[0], ts[1], ts[2]}, Hkv, 0,
+                              static_cast<const __nv_bfloat16*>(xv), {xs[0], xs[1], xs[2]}};
+    rt.B = B;
+    rt.S = G;
+    rt.D = D;
+    rt.pos = pos;
+    rt.pos0 = 0;
+    rt.src = src;
+    rt.nsrc = L;
+    rt.nx = NX;
+    rt.status = reinterpret_cast<int*>(ws);
+    star::rope_set_freq(rt, D, theta);
+    e = star::launch_rope(rt, 2, st);
+    if (e != cudaSuccess) return cuda_fail(e, "prefix table launch");
+  }
 
   star::AttnParams ap;
   memset(&ap, 0, sizeof ap);
   if ((s = map_token_major(&ap.tmQ, qrot, B, L, Hq, D)) != STAR_OK) return s;
   if ((s = map_cache(&ap.tmK, k_cache, B * Hkv, Lcap, L, D, 128)) != STAR_OK) return s;
   if ((s = map_cache(&ap.tmV, v_cache, B * Hkv, Lcap, L, D, 128)) != STAR_OK) return s;
+  if (ext && G > 0) {
+    if ((s = map_cache(&ap.tmKP, pk_buf, B * Hkv, G, G, D, 128)) != STAR_OK) return s;
+    if ((s = map_cache(&ap.tmVP, pv_buf, B * Hkv, G, G, D, 128)) != STAR_OK) return s;
+  }
   const int g = Hq / Hkv;
   ap.geom.B = B;
   ap.geom.Hq = Hq;
@@ -319,11 +383,14 @@ star_status star_phase1_encode(const void* q, const void* k, const void* v, void
   ap.geom.hpc = (g % 2 == 0) ? 2 : 1;
   ap.geom.L = L;
   ap.geom.b = block_len;
-  ap.geom.a = anchor_len;
+  ap.geom.a = ext ? 0 : anchor_len;
   ap.geom.n = ceil_div(L, block_len);
   ap.geom.T = 0;
   ap.geom.tail_len = 0;
   ap.mode = 0;
+  ap.ext = ext ? 1 : 0;
+  ap.bounds = ext ? bounds : nullptr;
+  ap.G = ext ? G : 0;
   const long long items = (long long)ap.geom.phase1_items();
   if (items > (1ll << 31) - 1) return fail(STAR_ERR_INVALID_ARG, "problem too large");
   ap.num_items = (int)items;
@@ -337,6 +404,31 @@ star_status star_phase1_encode(const void* q, const void* k, const void* v, void
   e = star::launch_attn(ap, D, st);
   if (e != cudaSuccess) return cuda_fail(e, "phase-1 attention launch");
   return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+star_status star_phase1_encode(const void* q, const void* k, const void* v, void* o, void* k_cache,
+                               void* v_cache, int Lcap, float* lse, int B, int L, int Hq, int Hkv,
+                               int D, int block_len, int anchor_len, double theta, void* workspace,
+                               size_t workspace_bytes, void* cuda_stream) {
+  return phase1_run(q, k, v, o, k_cache, v_cache, Lcap, lse, B, L, Hq, Hkv, D, block_len,
+                    anchor_len, false, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, theta,
+                    workspace, workspace_bytes, cuda_stream);
+}
+
+star_status star_phase1_encode_ext(const void* q, const void* k, const void* v, void* o,
+                                   void* k_cache, void* v_cache, int Lcap, float* lse, int B, int L,
+                                   int Hq, int Hkv, int D, int block_len, const int32_t* prefix_src,
+                                   const int32_t* prefix_pos, int G, const int32_t* prefix_bounds,
+                                   const void* extra_k, const void* extra_v, int n_extra,
+                                   double theta, void* workspace, size_t workspace_bytes,
+                                   void* cuda_stream) {
+  return phase1_run(q, k, v, o, k_cache, v_cache, Lcap, lse, B, L, Hq, Hkv, D, block_len, 0, true,
+                    prefix_src, prefix_pos, G, prefix_bounds, extra_k, extra_v, n_extra, theta,
+                    workspace, workspace_bytes, cuda_stream);
 }
 
 size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lcap, int block_len) {

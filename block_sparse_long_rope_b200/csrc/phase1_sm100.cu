@@ -109,11 +109,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
   uint64_t* o_full = p_full + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_full + 1);
   __shared__ volatile int abort_flag;
+  __shared__ KvSpan s_span[2];  // the KV spans this item visits, in order
+  __shared__ int s_nspan, s_nkv;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WorkItem w = (p.mode == 0) ? p.geom.phase1_item(blockIdx.x) : p.geom.phase2_item(blockIdx.x);
   const int hpc = p.geom.hpc;
-  const int nkv = w.ntiles();
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -130,6 +131,30 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     mbar_init(o_full, 1);
     fence_barrier_init();
     abort_flag = 0;
+    // span list: the item's own spans, or in ext mode the block's slice of
+    // the prefix table (clamped to the table; a slice outside it is recorded
+    // as a bounds error) and the own block
+    int ns = 0;
+    if (p.mode == 0 && p.ext) {
+      const int blk = w.q_lo / p.geom.b;
+      if (p.bounds) {
+        int gs = p.bounds[2 * blk], ge = p.bounds[2 * blk + 1];
+        if (gs < 0 || ge > p.G || ge < gs) {
+          atomicOr(p.status, kDevBounds);
+          gs = imin(imax(gs, 0), p.G);
+          ge = imin(imax(ge, gs), p.G);
+        }
+        if (ge > gs) s_span[ns++] = KvSpan{gs, ceil_div(ge - gs, kTileN), gs, ge, 0, 1};
+      }
+      s_span[ns++] = w.span[w.nspan - 1];  // own block, causal
+    } else {
+      for (int t = 0; t < w.nspan; ++t)
+        if (w.span[t].ntiles > 0) s_span[ns++] = w.span[t];
+    }
+    int nt = 0;
+    for (int t = 0; t < ns; ++t) nt += s_span[t].ntiles;
+    s_nspan = ns;
+    s_nkv = nt;
   }
   if (warp == 9) {
     tmem_alloc(tmem_slot, C::kTmemCols);
@@ -139,6 +164,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  const int nkv = s_nkv;
 
   if (warp == 8) {
     // ---------------------------------------------------------------- producer
@@ -146,6 +172,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
       prefetch_tmap(&p.tmQ);
       prefetch_tmap(&p.tmK);
       prefetch_tmap(&p.tmV);
+      if (p.ext && p.G > 0) {
+        prefetch_tmap(&p.tmKP);
+        prefetch_tmap(&p.tmVP);
+      }
       mbar_arrive_expect_tx(q_full, hpc * C::kTile);
       for (int x = 0; x < hpc; ++x)
 #pragma unroll
@@ -154,22 +184,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
                       w.slot0 + x, w.q_lo, w.b);
       const int bz = w.b * p.geom.Hkv + w.kvh;
       int issued_k = 0, issued_v = 0;
+      int csi = 0, cti = 0;  // span cursor
       for (int it = 0; it < nkv; ++it) {
         const int st = it % S, use = it / S;
-        int key0, lo, hi, causal;
-        w.tile(it, &key0, &lo, &hi, &causal);
+        const KvSpan& sp = s_span[csi];
+        const int key0 = sp.key0 + cti * kTileN;
+        const CUtensorMap* mk = sp.src ? &p.tmKP : &p.tmK;
+        const CUtensorMap* mv = sp.src ? &p.tmVP : &p.tmV;
+        if (++cti == sp.ntiles) {
+          ++csi;
+          cti = 0;
+        }
         if (use > 0 && !mbar_wait(&k_empty[st], (use - 1) & 1, &abort_flag, p.status)) break;
         mbar_arrive_expect_tx(&k_full[st], C::kTile);
 #pragma unroll
         for (int hd = 0; hd < D / 64; ++hd)
-          tma_load_3d(sm + C::kOffK + st * C::kTile + hd * C::kHalf, &p.tmK, &k_full[st], hd * 64,
+          tma_load_3d(sm + C::kOffK + st * C::kTile + hd * C::kHalf, mk, &k_full[st], hd * 64,
                       key0, bz);
         ++issued_k;
         if (use > 0 && !mbar_wait(&v_empty[st], (use - 1) & 1, &abort_flag, p.status)) break;
         mbar_arrive_expect_tx(&v_full[st], C::kTile);
 #pragma unroll
         for (int hd = 0; hd < D / 64; ++hd)
-          tma_load_3d(sm + C::kOffV + st * C::kTile + hd * C::kHalf, &p.tmV, &v_full[st], hd * 64,
+          tma_load_3d(sm + C::kOffV + st * C::kTile + hd * C::kHalf, mv, &v_full[st], hd * 64,
                       key0, bz);
         ++issued_v;
       }
@@ -253,6 +290,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
 
+    int csi = 0, cti = 0;  // span cursor
     for (int it = 0; it < nkv; ++it) {
       if (!mbar_wait(&s_full[x], it & 1, &abort_flag, p.status)) {
         ok = false;
@@ -266,8 +304,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
 #pragma unroll
       for (int q = 0; q < 4; ++q) reg_fence32(sr[q]);
 
-      int key0, lo, hi, causal;
-      w.tile(it, &key0, &lo, &hi, &causal);
+      const KvSpan& sp = s_span[csi];
+      const int key0 = sp.key0 + cti * kTileN, lo = sp.lo, hi = sp.hi, causal = sp.causal;
+      if (++cti == sp.ntiles) {
+        ++csi;
+        cti = 0;
+      }
       const bool full_vis =
           key0 >= lo && key0 + 128 <= hi && (!causal || key0 + 127 <= min_pos);
       if (!full_vis) {

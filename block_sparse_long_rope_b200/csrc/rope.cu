@@ -14,6 +14,12 @@
 // enough to move a peaked softmax's log-sum-exp by ~3e-2; correct rounding
 // makes the cache reproducible bit for bit.
 //
+// In gather mode the output token s takes its input row from an index
+// table (a context row or a given row) and is rotated at pos[s]: this builds
+// the gathered prefix table of the generalised Phase 1 (Pulsar's sink and
+// summaries keep their original global positions [pith 2607.20457, "What
+// carries the argument"]).
+//
 // One launch handles up to three jobs (Q, K, V of one call): blockIdx.z
 // selects the job. Each CTA covers kTokPerCta tokens of one job; it first
 // computes the (cos, sin) table of its tokens in shared memory, then streams
@@ -44,6 +50,18 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
   __shared__ double s_sin[kTokPerCta][64];
   __shared__ float f_cos[kTokPerCta][64];
   __shared__ float f_sin[kTokPerCta][64];
+  __shared__ int s_row[kTokPerCta];  // gather mode: source row, >= 0 in x, < 0 in x2
+  __shared__ int s_ok[kTokPerCta];
+  if (p.src) {
+    if (threadIdx.x < ntok) {
+      const int r = p.src[tok0 + threadIdx.x];
+      const bool ok = (r >= 0 && r < p.nsrc) || (r < 0 && r >= -p.nx);
+      s_row[threadIdx.x] = r;
+      s_ok[threadIdx.x] = ok;
+      if (!ok && blockIdx.z == 0) atomicOr(p.status, kDevBounds);
+    }
+    __syncthreads();
+  }
   if (job.rotate) {
     for (int e = threadIdx.x; e < ntok * half; e += blockDim.x) {
       int t = e / half, i = e % half;
@@ -65,8 +83,20 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
     int h = (u / cpr) % job.H;
     int t = u / (cpr * job.H);
     int s = tok0 + t;
-    const __nv_bfloat16* xr = job.x + b * job.xs[0] + s * job.xs[1] + h * job.xs[2];
     __nv_bfloat16* yr = job.y + b * job.ys[0] + s * job.ys[1] + h * job.ys[2];
+    const __nv_bfloat16* xr;
+    if (!p.src) {
+      xr = job.x + b * job.xs[0] + s * job.xs[1] + h * job.xs[2];
+    } else if (!s_ok[t]) {
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      *reinterpret_cast<uint4*>(yr + 8 * c) = z;
+      *reinterpret_cast<uint4*>(yr + half + 8 * c) = z;
+      continue;
+    } else {
+      const int r = s_row[t];
+      xr = (r >= 0) ? job.x + b * job.xs[0] + r * job.xs[1] + h * job.xs[2]
+                    : job.x2 + b * job.x2s[0] + (-1 - r) * job.x2s[1] + h * job.x2s[2];
+    }
     uint4 lo = *reinterpret_cast<const uint4*>(xr + 8 * c);
     uint4 hi = *reinterpret_cast<const uint4*>(xr + half + 8 * c);
     if (job.rotate) {

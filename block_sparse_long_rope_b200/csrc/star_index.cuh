@@ -38,6 +38,7 @@ __host__ __device__ __forceinline__ void phase1_row_ranges(int r, int b, int a, 
 // c <= p. Tiles start at key0 + kTileN * t, t in [0, ntiles).
 struct KvSpan {
   int key0, ntiles, lo, hi, causal;
+  int src;  // 0: the KV cache, 1: the gathered prefix table
 };
 
 // A unit of attention work: query rows [q_lo, q_hi) of one (batch, head
@@ -118,14 +119,14 @@ struct AttnGeom {
     w.pos_base = 0;
     w.split = -1;
     // own block: tiles aligned to the block start, up to the diagonal tile
-    const KvSpan own{s, j + 1, s, L, 1};
+    const KvSpan own{s, j + 1, s, L, 1, 0};
     if (i > 0 && a > 0) {
-      w.span[0] = KvSpan{0, ceil_div(a, kTileN), 0, a, 0};  // the anchor c_1
+      w.span[0] = KvSpan{0, ceil_div(a, kTileN), 0, a, 0, 0};  // the anchor c_1
       w.span[1] = own;
       w.nspan = 2;
     } else {
       w.span[0] = own;
-      w.span[1] = KvSpan{0, 0, 0, 0, 0};
+      w.span[1] = KvSpan{0, 0, 0, 0, 0, 0};
       w.nspan = 1;
     }
     return w;
@@ -148,15 +149,15 @@ struct AttnGeom {
     w.pos_base = L + tail_len;
     w.split = split;
     w.nspan = 1;
-    w.span[1] = KvSpan{0, 0, 0, 0, 0};
+    w.span[1] = KvSpan{0, 0, 0, 0, 0, 0};
     if (split < n) {
       int s = split * b, e = imin(s + b, L);
-      w.span[0] = KvSpan{s, ceil_div(e - s, kTileN), s, e, 0};
+      w.span[0] = KvSpan{s, ceil_div(e - s, kTileN), s, e, 0, 0};
     } else {
       // tail keys [L, L + tail_len + T); this tile's last row sits at
       // position L + tail_len + q_hi - 1
       int last = tail_len + w.q_hi;  // keys needed: [L, L + last)
-      w.span[0] = KvSpan{L, ceil_div(last, kTileN), L, L + tail_len + T, 1};
+      w.span[0] = KvSpan{L, ceil_div(last, kTileN), L, L + tail_len + T, 1, 0};
     }
     return w;
   }

@@ -19,12 +19,20 @@ struct RopeJob {
   long long ys[3];
   int H;
   int rotate;       // 0: plain copy (V into the cache)
+  const __nv_bfloat16* x2;  // gather mode: the given rows [B, nx, H, D]
+  long long x2s[3];
 };
 struct RopeParams {
   RopeJob job[3];
   int B, S, D;
   const int32_t* pos;  // nullable: position of token s is pos0 + s
   long long pos0;
+  // gather mode (src != nullptr): output token s reads row src[s] of x when
+  // 0 <= src[s] < nsrc, row -1 - src[s] of x2 when -nx <= src[s] < 0;
+  // any other index writes a zero row and sets kDevBounds in *status
+  const int32_t* src;
+  int nsrc, nx;
+  int* status;
   double inv_freq[64];  // theta^(-2i/D), i < D/2 (fp64, from the host)
 };
 // Fills out[0..63] with theta^(-2i/D) for i < D/2 (zero beyond).
@@ -37,6 +45,11 @@ struct AttnParams {
   CUtensorMap tmQ;  // rotated Q [B, rows, Hq, D]: dims {D, Hq, rows, B}, box {64, 1, 128, 1}
   CUtensorMap tmK;  // K cache [B*Hkv, Lvalid, D]: dims {D, Lvalid, B*Hkv}, box {64, 128, 1}
   CUtensorMap tmV;  // V cache, same shape as K
+  CUtensorMap tmKP;  // prefix table K (rotated) [B*Hkv, G, D] (ext mode, G > 0)
+  CUtensorMap tmVP;  // prefix table V
+  int ext;           // Phase 1 with a gathered prefix table (star_phase1_encode_ext)
+  const int32_t* bounds;  // device [n][2]: block i sees table rows [bounds[2i], bounds[2i+1])
+  int G;                  // prefix table rows
   AttnGeom geom;
   int mode;         // 0: Phase 1 (bf16 o, lse), 1: Phase 2 partials
   int num_items;

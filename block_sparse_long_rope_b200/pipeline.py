@@ -53,12 +53,40 @@ class StarLayer:
             lse2=torch.empty((B, Hq, Tmax), dtype=torch.float32, device=dev),
         )
 
+        self.prefix = None
+
+    def set_prefix(self, src, pos, bounds, extra_k=None, extra_v=None):
+        """Replace the Star anchor by a gathered prefix table (see prefix.py):
+        later encode calls run star_phase1_encode_ext with it. None restores
+        the anchor."""
+        if src is None:
+            self.prefix = None
+            return
+        w, dev = self.w, self.buf.o.device
+        t = [torch.as_tensor(x, dtype=torch.int32).contiguous().to(dev) for x in (src, pos, bounds)]
+        if t[2].shape != (w.n_blocks, 2):
+            raise ValueError(f"bounds must be [{w.n_blocks}, 2]")
+        G = t[0].numel()
+        ws = star.alloc_workspace(
+            star.star_phase1_ext_workspace_bytes(w.B, w.L, w.Hq, w.Hkv, w.D, G), dev)
+        self.prefix = (t[0], t[1], t[2], extra_k, extra_v, ws)
+
     def encode(self, q, k, v, with_lse=True):
         b = self.buf
-        star.star_phase1_encode(q, k, v, b.o, b.k_cache, b.v_cache, self.w.block_len,
-                                self.w.anchor_len, self.w.theta, b.ws1,
-                                lse=b.lse if with_lse else None)
+        lse = b.lse if with_lse else None
+        if self.prefix is None:
+            star.star_phase1_encode(q, k, v, b.o, b.k_cache, b.v_cache, self.w.block_len,
+                                    self.w.anchor_len, self.w.theta, b.ws1, lse=lse)
+        else:
+            src, pos, bounds, xk, xv, ws = self.prefix
+            star.star_phase1_encode_ext(q, k, v, b.o, b.k_cache, b.v_cache, self.w.block_len,
+                                        self.w.theta, ws, prefix_src=src, prefix_pos=pos,
+                                        prefix_bounds=bounds, extra_k=xk, extra_v=xv, lse=lse)
         return b.o
+
+    @property
+    def ws_phase1(self):
+        return self.buf.ws1 if self.prefix is None else self.prefix[5]
 
     def partial(self, q, k, v, tail_len):
         """Phase-2 partials of T = q.shape[1] new tokens; returns contiguous views

@@ -76,6 +76,51 @@ def star_phase1_encode(q, k, v, o, k_cache, v_cache, block_len, anchor_len, thet
     return o
 
 
+def star_phase1_ext_workspace_bytes(B, L, Hq, Hkv, D, G=0) -> int:
+    return int(_abi.load().star_phase1_ext_workspace_bytes(B, L, Hq, Hkv, D, G))
+
+
+def _i32(t, name):
+    if t is None:
+        return
+    if t.dtype != torch.int32 or not t.is_contiguous() or not t.is_cuda:
+        raise ValueError(f"{name} must be a contiguous int32 CUDA tensor")
+
+
+def star_phase1_encode_ext(q, k, v, o, k_cache, v_cache, block_len, theta, workspace,
+                           prefix_src=None, prefix_pos=None, prefix_bounds=None, extra_k=None,
+                           extra_v=None, lse=None, stream=None):
+    """Phase 1 with a gathered prefix table: row g is context row
+    prefix_src[g] (>= 0) or row -1 - prefix_src[g] of extra_k/extra_v
+    [B, NX, Hkv, D], its key rotated at prefix_pos[g]; block i sees table
+    rows prefix_bounds[i, 0] .. prefix_bounds[i, 1] - 1 (int32 [n, 2])."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _bf16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    B, L, Hq, D = q.shape
+    Hkv = k.shape[2]
+    Lcap = k_cache.shape[2]
+    for t, n in ((prefix_src, "prefix_src"), (prefix_pos, "prefix_pos"),
+                 (prefix_bounds, "prefix_bounds")):
+        _i32(t, n)
+    G = 0 if prefix_src is None else prefix_src.numel()
+    if prefix_pos is not None and prefix_pos.numel() != G:
+        raise ValueError("prefix_pos must have as many entries as prefix_src")
+    NX = 0
+    if extra_k is not None:
+        _bf16(extra_k, "extra_k")
+        _bf16(extra_v, "extra_v")
+        NX = extra_k.shape[1]
+    lib = _abi.load()
+    _abi.check(lib.star_phase1_encode_ext(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(k_cache), _ptr(v_cache), Lcap, _ptr(lse), B, L,
+        Hq, Hkv, D, int(block_len), _ptr(prefix_src), _ptr(prefix_pos), G, _ptr(prefix_bounds),
+        _ptr(extra_k), _ptr(extra_v), NX, float(theta), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o
+
+
 def star_phase2_workspace_bytes(B, T, Hq, Hkv, D, Lcap, block_len) -> int:
     return int(_abi.load().star_phase2_workspace_bytes(B, T, Hq, Hkv, D, Lcap, block_len))
 

@@ -112,6 +112,47 @@ star_status star_phase1_encode(const void* q, const void* k, const void* v, void
                                double theta, void* workspace, size_t workspace_bytes,
                                void* cuda_stream);
 
+/* Workspace bytes star_phase1_encode_ext needs for a prefix table of G
+ * rows: as star_phase1_encode plus the table's rotated K and its V (bf16
+ * [B, Hkv, G, D] each). */
+size_t star_phase1_ext_workspace_bytes(int B, int L, int Hq, int Hkv, int D, int G);
+
+/*
+ * star_phase1_encode_ext — Phase 1 with a generalised prefix. Instead of the
+ * anchor of star_phase1_encode, every block sees a slice of one gathered
+ * prefix table of G rows:
+ *   table row g  = context row prefix_src[g] of k/v when prefix_src[g] >= 0,
+ *                  row -1 - prefix_src[g] of extra_k/extra_v otherwise; its
+ *                  key is rotated at position prefix_pos[g];
+ *   block i sees table rows [prefix_bounds[2i], prefix_bounds[2i+1]), all
+ *                  visible, then its own rows causally at their own positions.
+ * This covers the Star anchor (rows 0..a-1 at positions 0..a-1, blocks i >= 1
+ * see [0, a)) [pith 2WVXFXZ2, "What carries the argument"]; the anchor
+ * ablations — no anchor, anchor position IDs moved or randomised, anchor
+ * content replaced (atlas.scime.ai summary, measured-effects table); and
+ * Pulsar's [sink || Sigma_0 || ... || Sigma_{i-1} || B_i] with every row at
+ * its original global position, one table of which block i sees a leading
+ * part [pith 2607.20457, "What carries the argument"]. A row listed twice
+ * counts twice; block 0 takes its slice too.
+ *
+ * prefix_src, prefix_pos : device int32 [G]; prefix_bounds: device int32
+ *   [n][2], n = ceil(L / block_len). All three may be NULL when G == 0.
+ * extra_k, extra_v : device bf16 [B, n_extra, Hkv, D] pre-RoPE, 16-byte
+ *   aligned; NULL when n_extra == 0.
+ * Other arguments, the outputs and the KV cache as for star_phase1_encode.
+ * Errors: invalid arguments as for star_phase1_encode (STAR_ERR_INVALID_ARG,
+ *   nothing launched). A prefix_src outside [-n_extra, L) gives a zero row; a
+ *   slice outside [0, G] (or reversed) is clamped to it; either records
+ *   STAR_ERR_DEVICE_BOUNDS in the workspace status word (star_device_status).
+ */
+star_status star_phase1_encode_ext(const void* q, const void* k, const void* v, void* o,
+                                   void* k_cache, void* v_cache, int Lcap, float* lse, int B, int L,
+                                   int Hq, int Hkv, int D, int block_len, const int32_t* prefix_src,
+                                   const int32_t* prefix_pos, int G, const int32_t* prefix_bounds,
+                                   const void* extra_k, const void* extra_v, int n_extra,
+                                   double theta, void* workspace, size_t workspace_bytes,
+                                   void* cuda_stream);
+
 /* Workspace bytes star_phase2_partial needs for up to T new tokens with a
  * cache of capacity Lcap (context L plus tail) split into blocks of
  * block_len. */

@@ -90,6 +90,43 @@ def test_phase1_validation(lib, kw, status):
     assert lib.star_last_error()  # a message is kept
 
 
+def test_ext_workspace_sizes(lib):
+    base = lib.star_phase1_workspace_bytes(1, 2048, 4, 64)
+    assert lib.star_phase1_ext_workspace_bytes(1, 2048, 4, 2, 64, 0) == base
+    # + the gathered table's K and V, bf16 [B, Hkv, G, D] each
+    assert lib.star_phase1_ext_workspace_bytes(1, 2048, 4, 2, 64, 100) == base + 2 * 100 * 2 * 64 * 2
+    assert lib.star_phase1_ext_workspace_bytes(1, 2048, 4, 2, 64, -1) == 256
+
+
+def _p1x(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, kc=FAKE, vc=FAKE, Lcap=64, lse=NULL, B=1, L=64,
+             Hq=4, Hkv=2, D=64, b=16, src=FAKE, pos=FAKE, G=8, bounds=FAKE, xk=NULL, xv=NULL,
+             NX=0, theta=1e4, ws=FAKE, wsb=1 << 30)
+    a.update(kw)
+    return lib.star_phase1_encode_ext(a["q"], a["k"], a["v"], a["o"], a["kc"], a["vc"], a["Lcap"],
+                                      a["lse"], a["B"], a["L"], a["Hq"], a["Hkv"], a["D"], a["b"],
+                                      a["src"], a["pos"], a["G"], a["bounds"], a["xk"], a["xv"],
+                                      a["NX"], a["theta"], a["ws"], a["wsb"], NULL)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(G=-1), INVALID),
+    (dict(src=NULL), INVALID),             # G > 0 needs the table
+    (dict(pos=NULL), INVALID),
+    (dict(bounds=NULL), INVALID),
+    (dict(src=ctypes.c_void_p(0x10002)), INVALID),
+    (dict(NX=-1), INVALID),
+    (dict(NX=2), INVALID),                 # extra rows without buffers
+    (dict(NX=2, xk=FAKE, xv=ODD), INVALID),
+    (dict(wsb=256 + 64 * 4 * 64 * 2), INVALID),  # room for Q only, not the table
+    (dict(D=96), UNSUPPORTED),
+    (dict(Lcap=63), INVALID),
+])
+def test_phase1_ext_validation(lib, kw, status):
+    assert _p1x(lib, **kw) == status
+    assert lib.star_last_error()
+
+
 def _p2(lib, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, T=1, kc=FAKE, vc=FAKE, Lcap=100, L=64, b=16, tail=0,
              po=FAKE, pl=FAKE, B=1, Hq=4, Hkv=2, D=64, theta=1e4, ws=FAKE, wsb=1 << 30)
@@ -134,6 +171,7 @@ def test_valid_call_without_device_reports_cuda_error(lib):
     # and the call returns an error instead of launching
     assert _p1(lib) in (CUDA, UNSUPPORTED)
     assert lib.star_last_error()
+    assert _p1x(lib, G=0, src=NULL, pos=NULL, bounds=NULL) in (CUDA, UNSUPPORTED)
 
 
 def test_python_binding_raises_on_missing_library(tmp_path):
