@@ -28,6 +28,8 @@ EXPORTS = (
     "star_phase1_encode",
     "star_phase1_ext_workspace_bytes",
     "star_phase1_encode_ext",
+    "star_phase2_partial_ext",
+    "star_lse_merge_ranks",
     "star_phase2_workspace_bytes",
     "star_phase2_partial",
     "star_phase2_decode_static",
@@ -84,7 +86,12 @@ def load(path: str = LIB_PATH):
         lib.star_phase1_ext_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I]
         lib.star_phase1_encode_ext.restype = _I
         lib.star_phase1_encode_ext.argtypes = [_P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I,
-                                               _I, _P, _P, _I, _P, _P, _P, _I, _D, _P, _SZ, _P]
+                                               _I, _P, _P, _I, _P, _P, _P, _I, _I, _D, _P, _SZ, _P]
+        lib.star_phase2_partial_ext.restype = _I
+        lib.star_phase2_partial_ext.argtypes = [_P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I,
+                                                _P, _P, _IP, _I, _I, _I, _I, _D, _P, _SZ, _P]
+        lib.star_lse_merge_ranks.restype = _I
+        lib.star_lse_merge_ranks.argtypes = [_P, _P, _I, _IP, _I, _P, _P, _I, _I, _I, _I, _P]
         lib.star_phase2_workspace_bytes.restype = _SZ
         lib.star_phase2_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I, _I]
         lib.star_phase2_partial.restype = _I

@@ -162,12 +162,12 @@ int decode_chunks_per_head(int L, int b, int n, int tail_plus_T, int chunk, int*
 // CTAs left after one extra unit per split for the ragged ends), and so that
 // a split has at most kMaxChunksPerSplit units. When there are more splits
 // than CTAs every split is one unit and CTAs loop over several.
-int decode_chunk(int B, int Hkv, int L, int b, int n, int tail_plus_T, int sms) {
+int decode_chunk(int B, int Hkv, int L, int b, int n, int nsplit, int tail_plus_T, int sms) {
   const int tile = star::kDecTile;
   const long long tiles_head = (long long)(n - 1) * ceil_div(imin(b, L), tile) +
                                ceil_div(L - (n - 1) * b, tile) + ceil_div(tail_plus_T, tile);
   const long long total_tiles = tiles_head * B * Hkv;
-  const long long splits = (long long)B * Hkv * (n + 1);
+  const long long splits = (long long)B * Hkv * nsplit;
   const long long ctas = 2ll * sms;
   const long long room = ctas - splits;
   const int max_split_tiles = ceil_div(star::imax(imin(b, L), tail_plus_T), tile);
@@ -270,7 +270,7 @@ star_status phase1_run(const void* q, const void* k, const void* v, void* o, voi
                        void* v_cache, int Lcap, float* lse, int B, int L, int Hq, int Hkv, int D,
                        int block_len, int anchor_len, bool ext, const int32_t* src,
                        const int32_t* pos, int G, const int32_t* bounds, const void* xk,
-                       const void* xv, int NX, double theta, void* workspace,
+                       const void* xv, int NX, int ctx_pos0, double theta, void* workspace,
                        size_t workspace_bytes, void* cuda_stream) {
   star_status s;
   if ((s = check_heads(B, Hq, Hkv, D)) != STAR_OK) return s;
@@ -291,6 +291,9 @@ star_status phase1_run(const void* q, const void* k, const void* v, void* o, voi
         return fail(STAR_ERR_INVALID_ARG, "prefix_bounds is NULL or not 4-byte aligned");
     }
     if (NX > 0 && ((s = check_ptr(xk, "extra_k")) || (s = check_ptr(xv, "extra_v")))) return s;
+    if (ctx_pos0 < 0 || (long long)ctx_pos0 + L > INT32_MAX)
+      return fail(STAR_ERR_INVALID_ARG, "ctx_pos0 (%d) must be >= 0 with ctx_pos0 + L in int32",
+                  ctx_pos0);
   }
   if (Lcap < L) return fail(STAR_ERR_INVALID_ARG, "Lcap (%d) < L (%d)", Lcap, L);
   if (!(theta > 0.0)) return fail(STAR_ERR_INVALID_ARG, "theta must be > 0");
@@ -336,7 +339,7 @@ star_status phase1_run(const void* q, const void* k, const void* v, void* o, voi
   rp.S = L;
   rp.D = D;
   rp.pos = nullptr;
-  rp.pos0 = 0;
+  rp.pos0 = ctx_pos0;  // context row r sits at ctx_pos0 + r
   star::rope_set_freq(rp, D, theta);
   e = star::launch_rope(rp, 3, st);
   if (e != cudaSuccess) return cuda_fail(e, "rope launch");
@@ -415,7 +418,7 @@ star_status star_phase1_encode(const void* q, const void* k, const void* v, void
                                int D, int block_len, int anchor_len, double theta, void* workspace,
                                size_t workspace_bytes, void* cuda_stream) {
   return phase1_run(q, k, v, o, k_cache, v_cache, Lcap, lse, B, L, Hq, Hkv, D, block_len,
-                    anchor_len, false, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, theta,
+                    anchor_len, false, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, 0, theta,
                     workspace, workspace_bytes, cuda_stream);
 }
 
@@ -424,11 +427,11 @@ star_status star_phase1_encode_ext(const void* q, const void* k, const void* v, 
                                    int Hq, int Hkv, int D, int block_len, const int32_t* prefix_src,
                                    const int32_t* prefix_pos, int G, const int32_t* prefix_bounds,
                                    const void* extra_k, const void* extra_v, int n_extra,
-                                   double theta, void* workspace, size_t workspace_bytes,
-                                   void* cuda_stream) {
+                                   int ctx_pos0, double theta, void* workspace,
+                                   size_t workspace_bytes, void* cuda_stream) {
   return phase1_run(q, k, v, o, k_cache, v_cache, Lcap, lse, B, L, Hq, Hkv, D, block_len, 0, true,
-                    prefix_src, prefix_pos, G, prefix_bounds, extra_k, extra_v, n_extra, theta,
-                    workspace, workspace_bytes, cuda_stream);
+                    prefix_src, prefix_pos, G, prefix_bounds, extra_k, extra_v, n_extra, ctx_pos0,
+                    theta, workspace, workspace_bytes, cuda_stream);
 }
 
 size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lcap, int block_len) {
@@ -444,26 +447,40 @@ size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lca
 
 namespace {
 
-// Body of star_phase2_partial / star_phase2_attend; o_merged == NULL skips the merge.
+// Body of star_phase2_partial / star_phase2_attend / star_phase2_partial_ext;
+// o_merged == NULL skips the merge. Cache row r sits at position ctx_pos0 + r,
+// new token t at q_pos0 + t. with_tail == 0: context splits only, nothing
+// appended (k, v unused).
 star_status phase2_run(const void* q, const void* k, const void* v, int T, void* k_cache,
-                       void* v_cache, int Lcap, int L, int block_len, int tail_len, float* part_o,
-                       float* part_lse, void* o_merged, float* lse_merged, int* nsplit_out, int B,
-                       int Hq, int Hkv, int D, double theta, void* workspace,
-                       size_t workspace_bytes, void* cuda_stream) {
+                       void* v_cache, int Lcap, int L, int block_len, int tail_len, int ctx_pos0,
+                       int q_pos0, int with_tail, float* part_o, float* part_lse, void* o_merged,
+                       float* lse_merged, int* nsplit_out, int B, int Hq, int Hkv, int D,
+                       double theta, void* workspace, size_t workspace_bytes, void* cuda_stream) {
   star_status s;
   if ((s = check_heads(B, Hq, Hkv, D)) != STAR_OK) return s;
   if (T < 1) return fail(STAR_ERR_INVALID_ARG, "T must be >= 1");
   if (L < 1) return fail(STAR_ERR_INVALID_ARG, "L must be >= 1");
   if (block_len < 1) return fail(STAR_ERR_INVALID_ARG, "block_len must be >= 1");
   if (tail_len < 0) return fail(STAR_ERR_INVALID_ARG, "tail_len must be >= 0");
-  if ((long long)L + tail_len + T > Lcap)
+  if (with_tail != 0 && with_tail != 1) return fail(STAR_ERR_INVALID_ARG, "with_tail must be 0 or 1");
+  if (!with_tail && tail_len != 0)
+    return fail(STAR_ERR_INVALID_ARG, "tail_len must be 0 without the tail split");
+  if (ctx_pos0 < 0 || q_pos0 < 0) return fail(STAR_ERR_INVALID_ARG, "positions must be >= 0");
+  if (with_tail && (long long)q_pos0 != (long long)ctx_pos0 + L + tail_len)
+    return fail(STAR_ERR_INVALID_ARG,
+                "with the tail split the new tokens follow the cache: q_pos0 (%d) != ctx_pos0 + L "
+                "+ tail_len (%lld)", q_pos0, (long long)ctx_pos0 + L + tail_len);
+  if ((long long)q_pos0 + T > INT32_MAX || (long long)ctx_pos0 + Lcap > INT32_MAX)
+    return fail(STAR_ERR_INVALID_ARG, "positions exceed int32");
+  if ((long long)L + tail_len + (with_tail ? T : 0) > Lcap)
     return fail(STAR_ERR_INVALID_ARG, "Lcap (%d) < L + tail_len + T (%lld)", Lcap,
-                (long long)L + tail_len + T);
+                (long long)L + tail_len + (with_tail ? T : 0));
   if (!(theta > 0.0)) return fail(STAR_ERR_INVALID_ARG, "theta must be > 0");
-  if ((s = check_ptr(q, "q")) || (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) ||
-      (s = check_ptr(k_cache, "k_cache")) || (s = check_ptr(v_cache, "v_cache")) ||
-      (s = check_ptr(part_o, "part_o")) || (s = check_ptr(workspace, "workspace")))
+  if ((s = check_ptr(q, "q")) || (s = check_ptr(k_cache, "k_cache")) ||
+      (s = check_ptr(v_cache, "v_cache")) || (s = check_ptr(part_o, "part_o")) ||
+      (s = check_ptr(workspace, "workspace")))
     return s;
+  if (with_tail && ((s = check_ptr(k, "k")) || (s = check_ptr(v, "v")))) return s;
   if (!part_lse || (reinterpret_cast<uintptr_t>(part_lse) & 3u))
     return fail(STAR_ERR_INVALID_ARG, "part_lse is NULL or not 4-byte aligned");
   if (o_merged && !aligned16(o_merged))
@@ -486,8 +503,8 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   cudaError_t e = cudaMemsetAsync(ws, 0, header, st);
   if (e != cudaSuccess) return cuda_fail(e, "status reset");
 
-  // RoPE of the new tokens at positions L + tail_len + t; K/V appended to the
-  // cache rows of the same index. The decode kernel does both itself.
+  // RoPE of the new tokens at positions q_pos0 + t; with the tail, K/V
+  // appended to cache rows L + tail_len + t. The decode kernel does both itself.
   const int row0 = L + tail_len;
   star::RopeParams rp{};
   const long long qs[3] = {(long long)T * Hq * D, (long long)Hq * D, D};
@@ -505,16 +522,16 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   rp.S = T;
   rp.D = D;
   rp.pos = nullptr;
-  rp.pos0 = row0;
+  rp.pos0 = q_pos0;
   star::rope_set_freq(rp, D, theta);
   if (!decode) {
-    e = star::launch_rope(rp, 3, st);
+    e = star::launch_rope(rp, with_tail ? 3 : 1, st);
     if (e != cudaSuccess) return cuda_fail(e, "rope launch");
   }
 
   const int n = ceil_div(L, block_len);
-  const int nsplit = n + 1;
-  const int valid = L + tail_len + T;
+  const int nsplit = n + with_tail;
+  const int valid = L + tail_len + (with_tail ? T : 0);
   const int g = Hq / Hkv;
   if (nsplit_out) *nsplit_out = nsplit;
 
@@ -540,9 +557,14 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
     dp.b = block_len;
     dp.n = n;
     dp.tail_len = tail_len;
-    const int chunk = decode_chunk(B, Hkv, L, block_len, n, tail_len + T, sms);
+    dp.ctx_pos0 = ctx_pos0;
+    dp.q_pos0 = q_pos0;
+    dp.with_tail = with_tail;
+    dp.nsplit = nsplit;
+    const int tail_rows = with_tail ? tail_len + T : 0;
+    const int chunk = decode_chunk(B, Hkv, L, block_len, n, nsplit, tail_rows, sms);
     dp.chunk = chunk;
-    dp.chunks_per_head = decode_chunks_per_head(L, block_len, n, tail_len + T, chunk, &dp.nc_full,
+    dp.chunks_per_head = decode_chunks_per_head(L, block_len, n, tail_rows, chunk, &dp.nc_full,
                                                 &dp.nc_last, &dp.nc_tail);
     const size_t rows = (size_t)B * Hkv * dp.chunks_per_head * star::kDecRows;
     dp.ws_o = reinterpret_cast<float*>(ws + header + qrot_bytes);
@@ -577,6 +599,7 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   ap.geom.n = n;
   ap.geom.T = T;
   ap.geom.tail_len = tail_len;
+  ap.geom.tail = with_tail;
   ap.mode = 1;
   ap.num_items = ap.geom.phase2_items();
   ap.qrows = T;
@@ -589,7 +612,11 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   e = star::launch_attn(ap, D, st);
   if (e != cudaSuccess) return cuda_fail(e, "phase-2 chunk attention launch");
   if (o_merged) {
-    e = star::launch_lse_merge(part_o, part_lse, nsplit, static_cast<__nv_bfloat16*>(o_merged),
+    star::MergeSegs segs{};
+    segs.nseg = 1;
+    segs.slots = nsplit;
+    segs.ns[0] = nsplit;
+    e = star::launch_lse_merge(part_o, part_lse, segs, static_cast<__nv_bfloat16*>(o_merged),
                                lse_merged, B, T, Hq, D, st);
     if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
   }
@@ -605,9 +632,9 @@ star_status star_phase2_partial(const void* q, const void* k, const void* v, int
                                 float* part_o, float* part_lse, int* nsplit_out, int B, int Hq,
                                 int Hkv, int D, double theta, void* workspace,
                                 size_t workspace_bytes, void* cuda_stream) {
-  return phase2_run(q, k, v, T, k_cache, v_cache, Lcap, L, block_len, tail_len, part_o, part_lse,
-                    nullptr, nullptr, nsplit_out, B, Hq, Hkv, D, theta, workspace,
-                    workspace_bytes, cuda_stream);
+  return phase2_run(q, k, v, T, k_cache, v_cache, Lcap, L, block_len, tail_len, 0, L + tail_len,
+                    1, part_o, part_lse, nullptr, nullptr, nsplit_out, B, Hq, Hkv, D, theta,
+                    workspace, workspace_bytes, cuda_stream);
 }
 
 star_status star_phase2_attend(const void* q, const void* k, const void* v, int T, void* k_cache,
@@ -616,9 +643,20 @@ star_status star_phase2_attend(const void* q, const void* k, const void* v, int 
                                int* nsplit_out, int B, int Hq, int Hkv, int D, double theta,
                                void* workspace, size_t workspace_bytes, void* cuda_stream) {
   if (!o) return fail(STAR_ERR_INVALID_ARG, "o is NULL");
-  return phase2_run(q, k, v, T, k_cache, v_cache, Lcap, L, block_len, tail_len, part_o, part_lse,
-                    o, lse, nsplit_out, B, Hq, Hkv, D, theta, workspace, workspace_bytes,
-                    cuda_stream);
+  return phase2_run(q, k, v, T, k_cache, v_cache, Lcap, L, block_len, tail_len, 0, L + tail_len,
+                    1, part_o, part_lse, o, lse, nsplit_out, B, Hq, Hkv, D, theta, workspace,
+                    workspace_bytes, cuda_stream);
+}
+
+star_status star_phase2_partial_ext(const void* q, const void* k, const void* v, int T,
+                                    void* k_cache, void* v_cache, int Lcap, int L, int block_len,
+                                    int tail_len, int ctx_pos0, int q_pos0, int with_tail,
+                                    float* part_o, float* part_lse, int* nsplit_out, int B, int Hq,
+                                    int Hkv, int D, double theta, void* workspace,
+                                    size_t workspace_bytes, void* cuda_stream) {
+  return phase2_run(q, k, v, T, k_cache, v_cache, Lcap, L, block_len, tail_len, ctx_pos0, q_pos0,
+                    with_tail, part_o, part_lse, nullptr, nullptr, nsplit_out, B, Hq, Hkv, D,
+                    theta, workspace, workspace_bytes, cuda_stream);
 }
 
 star_status star_lse_merge(const float* part_o, const float* part_lse, int nsplit, void* o,
@@ -633,7 +671,47 @@ star_status star_lse_merge(const float* part_o, const float* part_lse, int nspli
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
     return fail(STAR_ERR_INVALID_ARG, "lse is not 4-byte aligned");
   if ((s = check_device(nullptr)) != STAR_OK) return s;
-  cudaError_t e = star::launch_lse_merge(part_o, part_lse, nsplit, static_cast<__nv_bfloat16*>(o),
+  star::MergeSegs segs{};
+  segs.nseg = 1;
+  segs.slots = nsplit;
+  segs.ns[0] = nsplit;
+  cudaError_t e = star::launch_lse_merge(part_o, part_lse, segs, static_cast<__nv_bfloat16*>(o),
+                                         lse, B, T, Hq, D, static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
+  return ok();
+}
+
+star_status star_lse_merge_ranks(const float* part_o, const float* part_lse, int nranks,
+                                 const int* nsplit_of_rank, int nsplit_stride, void* o, float* lse,
+                                 int B, int T, int Hq, int D, void* cuda_stream) {
+  if (nranks < 1 || nranks > star::kMaxMergeSegs)
+    return fail(STAR_ERR_INVALID_ARG, "nranks (%d) must lie in [1, %d]", nranks,
+                star::kMaxMergeSegs);
+  if (!nsplit_of_rank) return fail(STAR_ERR_INVALID_ARG, "nsplit_of_rank is NULL");
+  if (nsplit_stride < 1 || B < 1 || T < 1 || Hq < 1)
+    return fail(STAR_ERR_INVALID_ARG, "bad shape stride=%d B=%d T=%d Hq=%d", nsplit_stride, B, T,
+                Hq);
+  if (D != 64 && D != 128) return fail(STAR_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", D);
+  star::MergeSegs segs{};
+  segs.nseg = nranks;
+  segs.slots = nsplit_stride;
+  long long total = 0;
+  for (int r = 0; r < nranks; ++r) {
+    if (nsplit_of_rank[r] < 0 || nsplit_of_rank[r] > nsplit_stride)
+      return fail(STAR_ERR_INVALID_ARG, "rank %d has %d splits (stride %d)", r, nsplit_of_rank[r],
+                  nsplit_stride);
+    segs.ns[r] = nsplit_of_rank[r];
+    total += nsplit_of_rank[r];
+  }
+  if (total < 1) return fail(STAR_ERR_INVALID_ARG, "no splits to merge");
+  star_status s;
+  if ((s = check_ptr(part_o, "part_o")) || (s = check_ptr(o, "o"))) return s;
+  if (!part_lse || (reinterpret_cast<uintptr_t>(part_lse) & 3u))
+    return fail(STAR_ERR_INVALID_ARG, "part_lse is NULL or not 4-byte aligned");
+  if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+    return fail(STAR_ERR_INVALID_ARG, "lse is not 4-byte aligned");
+  if ((s = check_device(nullptr)) != STAR_OK) return s;
+  cudaError_t e = star::launch_lse_merge(part_o, part_lse, segs, static_cast<__nv_bfloat16*>(o),
                                          lse, B, T, Hq, D, static_cast<cudaStream_t>(cuda_stream));
   if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
   return ok();

@@ -8,6 +8,11 @@
 // which reproduces softmax over the concatenated keys exactly [pith 2WVXFXZ2,
 // assumptions: online softmax aggregation yields the exact global softmax].
 //
+// The splits may come in segments, one per rank after an all-gather of the
+// ranks' partials: segment s occupies B * Hq * slots split rows and begins
+// with its segs.ns[s] splits laid out [B, Hq, ns[s], T, D]. One segment with
+// slots = ns[0] = nsplit is the plain [B, Hq, nsplit, T, D] layout.
+//
 // One warp per (batch, head, token) row; lanes cover D with 16-byte loads.
 // HBM-bound and tiny: it reads nsplit * (D + 1) floats per row.
 #include <math.h>
@@ -20,7 +25,8 @@ namespace star {
 template <int D>
 __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict__ part_o,
                                                         const float* __restrict__ part_lse,
-                                                        int nsplit, __nv_bfloat16* __restrict__ o,
+                                                        const __grid_constant__ MergeSegs segs,
+                                                        __nv_bfloat16* __restrict__ o,
                                                         float* __restrict__ lse, int B, int T,
                                                         int Hq) {
   constexpr int kPer = D / 32;  // floats per lane (2 or 4)
@@ -32,40 +38,46 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict_
   const int h = (warp / T) % Hq;
   const int b = warp / (T * Hq);
   const size_t bh = static_cast<size_t>(b) * Hq + h;
+  const size_t seg_rows = static_cast<size_t>(B) * Hq * segs.slots;  // (b, h, split) rows per segment
+  auto split_row = [&](int seg, int s) { return (seg * seg_rows + bh * segs.ns[seg] + s) * T + t; };
 
   // statistics: lanes read the split LSEs in parallel, shuffles reduce them
   float m = -INFINITY;
-  for (int s = lane; s < nsplit; s += 32) m = fmaxf(m, part_lse[(bh * nsplit + s) * T + t]);
+  for (int seg = 0; seg < segs.nseg; ++seg)
+    for (int s = lane; s < segs.ns[seg]; s += 32) m = fmaxf(m, part_lse[split_row(seg, s)]);
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
   float acc[kPer];
 #pragma unroll
   for (int j = 0; j < kPer; ++j) acc[j] = 0.f;
   float z = 0.f;
   if (m != -INFINITY) {
-    for (int s0 = 0; s0 < nsplit; s0 += 32) {
-      const int sl = s0 + lane;
-      const float l = (sl < nsplit) ? part_lse[(bh * nsplit + sl) * T + t] : -INFINITY;
-      const float wl = (l == -INFINITY) ? 0.f : expf(l - m);
-      float zs = wl;
+    for (int seg = 0; seg < segs.nseg; ++seg) {
+      const int nsplit = segs.ns[seg];
+      for (int s0 = 0; s0 < nsplit; s0 += 32) {
+        const int sl = s0 + lane;
+        const float l = (sl < nsplit) ? part_lse[split_row(seg, sl)] : -INFINITY;
+        const float wl = (l == -INFINITY) ? 0.f : expf(l - m);
+        float zs = wl;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, o);
-      z += zs;
-      const int ns = imin(32, nsplit - s0);
+        for (int off = 16; off > 0; off >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, off);
+        z += zs;
+        const int ns = imin(32, nsplit - s0);
 #pragma unroll 4
-      for (int k = 0; k < ns; ++k) {  // independent loads: the weights are already known
-        const float w = __shfl_sync(0xffffffffu, wl, k);
-        const float* src = part_o + ((bh * nsplit + s0 + k) * T + t) * D + lane * kPer;
-        if constexpr (kPer == 4) {
-          const float4 v = *reinterpret_cast<const float4*>(src);
-          acc[0] += w * v.x;
-          acc[1] += w * v.y;
-          acc[2] += w * v.z;
-          acc[3] += w * v.w;
-        } else {
-          const float2 v = *reinterpret_cast<const float2*>(src);
-          acc[0] += w * v.x;
-          acc[1] += w * v.y;
+        for (int k = 0; k < ns; ++k) {  // independent loads: the weights are already known
+          const float w = __shfl_sync(0xffffffffu, wl, k);
+          const float* src = part_o + split_row(seg, s0 + k) * D + lane * kPer;
+          if constexpr (kPer == 4) {
+            const float4 v = *reinterpret_cast<const float4*>(src);
+            acc[0] += w * v.x;
+            acc[1] += w * v.y;
+            acc[2] += w * v.z;
+            acc[3] += w * v.w;
+          } else {
+            const float2 v = *reinterpret_cast<const float2*>(src);
+            acc[0] += w * v.x;
+            acc[1] += w * v.y;
+          }
         }
       }
     }
@@ -83,7 +95,7 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict_
   if (lse != nullptr && lane == 0) lse[bh * T + t] = (z > 0.f) ? m + logf(z) : -INFINITY;
 }
 
-cudaError_t launch_lse_merge(const float* part_o, const float* part_lse, int nsplit,
+cudaError_t launch_lse_merge(const float* part_o, const float* part_lse, const MergeSegs& segs,
                              __nv_bfloat16* o, float* lse, int B, int T, int Hq, int D,
                              cudaStream_t stream) {
   const long long rows = static_cast<long long>(B) * Hq * T;
@@ -91,11 +103,9 @@ cudaError_t launch_lse_merge(const float* part_o, const float* part_lse, int nsp
   const int threads = 256;
   const unsigned blocks = static_cast<unsigned>((rows * 32 + threads - 1) / threads);
   if (D == 128)
-    lse_merge_kernel<128><<<blocks, threads, 0, stream>>>(part_o, part_lse, nsplit, o, lse, B, T,
-                                                          Hq);
+    lse_merge_kernel<128><<<blocks, threads, 0, stream>>>(part_o, part_lse, segs, o, lse, B, T, Hq);
   else
-    lse_merge_kernel<64><<<blocks, threads, 0, stream>>>(part_o, part_lse, nsplit, o, lse, B, T,
-                                                         Hq);
+    lse_merge_kernel<64><<<blocks, threads, 0, stream>>>(part_o, part_lse, segs, o, lse, B, T, Hq);
   return cudaGetLastError();
 }
 

@@ -226,6 +226,10 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
   dp.b = block_len;
   dp.n = n;
   dp.tail_len = tail_len;
+  dp.ctx_pos0 = 0;
+  dp.q_pos0 = L + tail_len;
+  dp.with_tail = 1;
+  dp.nsplit = n + 1;
   dp.chunk = chunk;
   dp.chunks_per_head = chunks_per_head(L, block_len, n, tail_len + T, chunk, &dp.nc_full,
                                        &dp.nc_last, &dp.nc_tail);

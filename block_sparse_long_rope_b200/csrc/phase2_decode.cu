@@ -140,7 +140,7 @@ template <int D>
 __device__ void reduce_split(const DecodeParams& p, int bh, int split, float* sw) {
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
   constexpr int kC = kMaxChunksPerSplit;
-  const int nsplit = p.n + 1;
+  const int nsplit = p.nsplit;
   int first, count;
   split_chunks(p, split, &first, &count);
   const size_t cbase = static_cast<size_t>(bh) * p.chunks_per_head + first;
@@ -205,7 +205,7 @@ __device__ void reduce_split(const DecodeParams& p, int bh, int split, float* sw
 template <int D>
 __device__ void merge_head(const DecodeParams& p, int bh, float* sw) {
   const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int nsplit = p.n + 1;
+  const int nsplit = p.nsplit;
   const int b = bh / p.Hkv, kvh = bh % p.Hkv;
   float* rowm = sw;             // [R]
   float* rowz = sw + kDecRows;  // [R]
@@ -319,7 +319,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
       prefetch_tmap(&p.tmK);
       prefetch_tmap(&p.tmV);
     }
-    const int row0 = p.L + p.tail_len;  // cache row (= position) of new token 0
+    const int row0 = p.L + p.tail_len;  // cache row of new token 0
     int gt = 0;  // tiles issued over all units of this CTA
     bool stop = false;
     for (int u = u_begin; u < u_end && !stop; ++u) {
@@ -330,7 +330,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
       // row rotates its key and appends key and value before loading that
       // tile (no other unit reads the row). The warp writes, every lane
       // fences its generic writes against the TMA (async proxy) reads.
-      const int w_lo = imax(cr.k_lo, row0), w_hi = imin(cr.k_hi, row0 + p.T);
+      const int w_lo = imax(cr.k_lo, row0), w_hi = p.with_tail ? imin(cr.k_hi, row0 + p.T) : 0;
       if (w_lo < w_hi) {
         const int b = bh / p.Hkv, kvh = bh % p.Hkv;
         for (int r = w_lo; r < w_hi; ++r) {
@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
           __nv_bfloat16* vd = p.v_cache + (static_cast<size_t>(bh) * p.Lcap + r) * D;
           for (int i = lane; i < D / 2; i += 32) {
             double c64, s64;
-            rope_angle(r, p.inv_freq[i], &c64, &s64);
+            rope_angle(static_cast<long long>(p.ctx_pos0) + r, p.inv_freq[i], &c64, &s64);
             const float a = __bfloat162float(ks[i]), bb = __bfloat162float(ks[i + D / 2]);
             const float c32 = static_cast<float>(c64), s32 = static_cast<float>(s64);
             kd[i] = __ushort_as_bfloat16(static_cast<unsigned short>(rope_rotate_bf16(a, bb, c32, s32, c64, s64, true)));
@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
             const __nv_bfloat16* src =
                 p.q_new + ((static_cast<size_t>(b) * p.T + t) * p.Hq + kvh * g + hh) * D;
             double c64, s64;
-            rope_angle(p.L + p.tail_len + t, p.inv_freq[i], &c64, &s64);
+            rope_angle(static_cast<long long>(p.q_pos0) + t, p.inv_freq[i], &c64, &s64);
             const float a = __bfloat162float(src[i]), bb = __bfloat162float(src[i + D / 2]);
             const float c32 = static_cast<float>(c64), s32 = static_cast<float>(s64);
             y0 = rope_rotate_bf16(a, bb, c32, s32, c64, s64, true);
@@ -434,7 +434,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
 #pragma unroll
       for (int dn = 0; dn < D / 8; ++dn) o[dn][0] = o[dn][1] = o[dn][2] = o[dn][3] = 0.f;
       float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-      const int pos0 = p.L + p.tail_len + r0 / g;  // query positions of this thread's rows
+      const int pos0 = p.L + p.tail_len + r0 / g;  // cache rows of this thread's query tokens
       const int pos1 = p.L + p.tail_len + r1 / g;
 
       for (int it = 0; it < nt; ++it, ++gt) {
@@ -598,7 +598,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
         int first, count;
         split_chunks(p, cr.split, &first, &count);
         __threadfence();
-        flag_last = (atomicAdd(&p.counters[bh * (p.n + 1) + cr.split], 1) == count - 1);
+        flag_last = (atomicAdd(&p.counters[bh * p.nsplit + cr.split], 1) == count - 1);
         __threadfence();
       }
       consumer_sync();

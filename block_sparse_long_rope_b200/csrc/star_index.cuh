@@ -72,6 +72,7 @@ struct AttnGeom {
   int n;                // context blocks = ceil(L / b)
   // Phase 2 only
   int T, tail_len;
+  int tail;             // 1: the call's cache holds the tail split (new tokens)
 
   __host__ __device__ int groups() const { return B * Hkv * ((Hq / Hkv) / hpc); }
   __host__ __device__ int qtiles_full() const { return ceil_div(imin(b, L), kTileM); }
@@ -136,7 +137,7 @@ struct AttnGeom {
   // Items: split-major (context blocks 0..n-1, then the tail), then query
   // tile, then head group.
   __host__ __device__ int phase2_qtiles() const { return ceil_div(T, kTileM); }
-  __host__ __device__ int phase2_items() const { return (n + 1) * phase2_qtiles() * groups(); }
+  __host__ __device__ int phase2_items() const { return (n + tail) * phase2_qtiles() * groups(); }
   __host__ __device__ WorkItem phase2_item(int item) const {
     int G = groups(), nq = phase2_qtiles();
     int split = item / (nq * G);

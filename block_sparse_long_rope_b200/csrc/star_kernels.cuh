@@ -82,16 +82,20 @@ struct DecodeParams {
   double inv_freq[64];         // theta^(-2i/D), i < D/2
   int B, T, Hq, Hkv, g, R;  // R = T * g rows (<= kDecRows)
   int L, b, n, tail_len;    // context, block length, context splits, earlier tail tokens
+  int ctx_pos0;             // position of cache row 0 (row r sits at ctx_pos0 + r)
+  int q_pos0;               // position of new token 0
+  int with_tail;            // 1: append the new tokens and attend the tail split
+  int nsplit;               // n + with_tail
   int chunk;                // keys per CTA (multiple of kDecTile)
   int nc_full, nc_last, nc_tail, chunks_per_head;  // chunk counts per split kind
   float* ws_o;     // [B*Hkv, chunks_per_head, kDecRows, D] chunk-normalised output
   float* ws_lse;   // [B*Hkv, chunks_per_head, kDecRows]
-  int* counters;   // [B*Hkv, n+1] finished chunks per split, zero at launch
+  int* counters;   // [B*Hkv, nsplit] finished chunks per split, zero at launch
   int* head_counters;  // [B*Hkv] finished splits per (batch, KV head), zero at launch
   __nv_bfloat16* o_merged;  // nullable: [B, T, Hq, D] merged output (also needs head_counters)
   float* lse_merged;        // nullable: [B, Hq, T]
-  float* part_o;   // [B, Hq, n+1, T, D]
-  float* part_lse; // [B, Hq, n+1, T]
+  float* part_o;   // [B, Hq, nsplit, T, D]
+  float* part_lse; // [B, Hq, nsplit, T]
   int* status;
   float scale_log2, scale_ln;
 };
@@ -99,7 +103,15 @@ size_t decode_smem_bytes(int D);
 cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t stream);
 
 // ---- LSE merge ---------------------------------------------------------------
-cudaError_t launch_lse_merge(const float* part_o, const float* part_lse, int nsplit,
+// Partials in `nseg` segments (e.g. one per rank after an all-gather):
+// segment s starts at split row s * B * Hq * slots and holds its ns[s] <=
+// slots splits laid out densely, [B, Hq, ns[s], T, D] / [B, Hq, ns[s], T].
+constexpr int kMaxMergeSegs = 64;
+struct MergeSegs {
+  int nseg, slots;
+  int ns[kMaxMergeSegs];
+};
+cudaError_t launch_lse_merge(const float* part_o, const float* part_lse, const MergeSegs& segs,
                              __nv_bfloat16* o, float* lse, int B, int T, int Hq, int D,
                              cudaStream_t stream);
 

@@ -89,7 +89,7 @@ def _i32(t, name):
 
 def star_phase1_encode_ext(q, k, v, o, k_cache, v_cache, block_len, theta, workspace,
                            prefix_src=None, prefix_pos=None, prefix_bounds=None, extra_k=None,
-                           extra_v=None, lse=None, stream=None):
+                           extra_v=None, lse=None, ctx_pos0=0, stream=None):
     """Phase 1 with a gathered prefix table: row g is context row
     prefix_src[g] (>= 0) or row -1 - prefix_src[g] of extra_k/extra_v
     [B, NX, Hkv, D], its key rotated at prefix_pos[g]; block i sees table
@@ -116,7 +116,7 @@ def star_phase1_encode_ext(q, k, v, o, k_cache, v_cache, block_len, theta, works
     _abi.check(lib.star_phase1_encode_ext(
         _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(k_cache), _ptr(v_cache), Lcap, _ptr(lse), B, L,
         Hq, Hkv, D, int(block_len), _ptr(prefix_src), _ptr(prefix_pos), G, _ptr(prefix_bounds),
-        _ptr(extra_k), _ptr(extra_v), NX, float(theta), _ptr(workspace),
+        _ptr(extra_k), _ptr(extra_v), NX, int(ctx_pos0), float(theta), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _stream(stream)))
     return o
 
@@ -142,6 +142,31 @@ def star_phase2_partial(q, k, v, k_cache, v_cache, L, block_len, tail_len, part_
     _abi.check(lib.star_phase2_partial(
         _ptr(q), _ptr(k), _ptr(v), T, _ptr(k_cache), _ptr(v_cache), Lcap, int(L), int(block_len),
         int(tail_len), _ptr(part_o), _ptr(part_lse), ctypes.byref(ns), B, Hq, Hkv, D,
+        float(theta), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return ns.value
+
+
+def star_phase2_partial_ext(q, k, v, k_cache, v_cache, L, block_len, tail_len, ctx_pos0, q_pos0,
+                            with_tail, part_o, part_lse, theta, workspace, stream=None):
+    """Phase-2 partials of one shard: cache row r at position ctx_pos0 + r,
+    new token t at q_pos0 + t. with_tail: append k/v and add the tail split
+    (q_pos0 must be ctx_pos0 + L + tail_len); otherwise context splits only
+    (k, v may be None). Returns nsplit."""
+    for t, n in ((q, "q"), (k_cache, "k_cache"), (v_cache, "v_cache")) + \
+            (((k, "k"), (v, "v")) if with_tail else ()):
+        _bf16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    B, T, Hq, D = q.shape
+    Hkv = k_cache.shape[1]
+    Lcap = k_cache.shape[2]
+    ns = ctypes.c_int(0)
+    lib = _abi.load()
+    _abi.check(lib.star_phase2_partial_ext(
+        _ptr(q), _ptr(k if with_tail else None), _ptr(v if with_tail else None), T, _ptr(k_cache),
+        _ptr(v_cache), Lcap, int(L), int(block_len), int(tail_len), int(ctx_pos0), int(q_pos0),
+        1 if with_tail else 0, _ptr(part_o), _ptr(part_lse), ctypes.byref(ns), B, Hq, Hkv, D,
         float(theta), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)))
     return ns.value
@@ -195,6 +220,24 @@ def star_lse_merge(part_o, part_lse, o, lse=None, stream=None):
     lib = _abi.load()
     _abi.check(lib.star_lse_merge(_ptr(part_o), _ptr(part_lse), S, _ptr(o), _ptr(lse), B, T, Hq,
                                   D, _stream(stream)))
+    return o
+
+
+def star_lse_merge_ranks(part_o, part_lse, nsplit_of_rank, slots, o, lse=None, stream=None):
+    """Merge partials gathered from ranks: part_o / part_lse hold one slot of
+    B*Hq*slots*T*D / B*Hq*slots*T floats per rank, rank r's slot beginning
+    with its [B, Hq, nsplit_of_rank[r], T, (D)] partials -> o[B,T,Hq,D]
+    bf16, lse[B,Hq,T]."""
+    B, T, Hq, D = o.shape
+    R = len(nsplit_of_rank)
+    S = int(slots)
+    if part_o.numel() < R * B * Hq * S * T * D or part_lse.numel() < R * B * Hq * S * T:
+        raise ValueError("gathered buffers smaller than nranks slots")
+    _bf16(o, "o")
+    ns = (ctypes.c_int * R)(*[int(x) for x in nsplit_of_rank])
+    lib = _abi.load()
+    _abi.check(lib.star_lse_merge_ranks(_ptr(part_o), _ptr(part_lse), R, ns, S, _ptr(o), _ptr(lse),
+                                        B, T, Hq, D, _stream(stream)))
     return o
 
 

@@ -139,6 +139,12 @@ size_t star_phase1_ext_workspace_bytes(int B, int L, int Hq, int Hkv, int D, int
  *   [n][2], n = ceil(L / block_len). All three may be NULL when G == 0.
  * extra_k, extra_v : device bf16 [B, n_extra, Hkv, D] pre-RoPE, 16-byte
  *   aligned; NULL when n_extra == 0.
+ * ctx_pos0 : position of context row 0 (row r of q/k/v sits at ctx_pos0 + r;
+ *   0 for a whole sequence). A shard of a sequence split by blocks over
+ *   several GPUs passes the global position of its first row, with the
+ *   anchor as given rows at positions 0..a-1 [pith 2WVXFXZ2, "What carries
+ *   the argument": every host gets the anchor block with its original
+ *   positions]. Block boundaries are counted from row 0 of the call.
  * Other arguments, the outputs and the KV cache as for star_phase1_encode.
  * Errors: invalid arguments as for star_phase1_encode (STAR_ERR_INVALID_ARG,
  *   nothing launched). A prefix_src outside [-n_extra, L) gives a zero row; a
@@ -150,8 +156,8 @@ star_status star_phase1_encode_ext(const void* q, const void* k, const void* v, 
                                    int Hq, int Hkv, int D, int block_len, const int32_t* prefix_src,
                                    const int32_t* prefix_pos, int G, const int32_t* prefix_bounds,
                                    const void* extra_k, const void* extra_v, int n_extra,
-                                   double theta, void* workspace, size_t workspace_bytes,
-                                   void* cuda_stream);
+                                   int ctx_pos0, double theta, void* workspace,
+                                   size_t workspace_bytes, void* cuda_stream);
 
 /* Workspace bytes star_phase2_partial needs for up to T new tokens with a
  * cache of capacity Lcap (context L plus tail) split into blocks of
@@ -200,6 +206,34 @@ star_status star_phase2_attend(const void* q, const void* k, const void* v, int 
                                void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
+ * star_phase2_partial_ext — star_phase2_partial for one shard of a sequence
+ * whose context blocks are spread over several GPUs [pith 2WVXFXZ2, Referee
+ * summary: the query is broadcast, every host computes a local attention
+ * output and softmax statistic over its own KV cache, the query host
+ * re-weights them; "What carries the argument": KV caches never move].
+ *   cache row r (r < L + tail_len) sits at position ctx_pos0 + r;
+ *   new token t is rotated at position q_pos0 + t;
+ *   with_tail = 1 (the query host): as star_phase2_partial — the new tokens'
+ *     k/v are rotated and appended at cache rows L + tail_len + t, which
+ *     requires q_pos0 == ctx_pos0 + L + tail_len, and split n is the causal
+ *     tail; nsplit = n + 1;
+ *   with_tail = 0 (any other host): context splits only; k and v are unused
+ *     (may be NULL), tail_len must be 0, nothing is written to the cache;
+ *     nsplit = n.
+ * n = ceil(L / block_len) counts the shard's own blocks. part_o [B, Hq,
+ * nsplit, T, D] and part_lse [B, Hq, nsplit, T] fp32 as star_phase2_partial.
+ * Workspace: star_phase2_workspace_bytes(B, T, Hq, Hkv, D, Lcap, block_len).
+ * Errors: STAR_ERR_INVALID_ARG for negative positions, with_tail not 0/1,
+ * q_pos0 inconsistent with the tail, or positions past int32.
+ */
+star_status star_phase2_partial_ext(const void* q, const void* k, const void* v, int T,
+                                    void* k_cache, void* v_cache, int Lcap, int L, int block_len,
+                                    int tail_len, int ctx_pos0, int q_pos0, int with_tail,
+                                    float* part_o, float* part_lse, int* nsplit_out, int B, int Hq,
+                                    int Hkv, int D, double theta, void* workspace,
+                                    size_t workspace_bytes, void* cuda_stream);
+
+/*
  * star_lse_merge — exact merge of per-split partials into global attention
  * [pith 2WVXFXZ2, minor comment on Algorithm 2 (corrected update
  * exp(s_h - s_global) * A_h); assumptions: online softmax aggregation gives
@@ -212,6 +246,21 @@ star_status star_phase2_attend(const void* q, const void* k, const void* v, int 
  */
 star_status star_lse_merge(const float* part_o, const float* part_lse, int nsplit, void* o,
                            float* lse, int B, int T, int Hq, int D, void* cuda_stream);
+
+/*
+ * star_lse_merge_ranks — star_lse_merge over partials gathered from several
+ * ranks (the query host's aggregation step [pith 2WVXFXZ2, Referee summary]).
+ * Every rank owns an equal slot of B * Hq * nsplit_stride * T * D floats of
+ * part_o and B * Hq * nsplit_stride * T floats of part_lse (an all-gather of
+ * equal-sized send buffers); rank r's slot begins with its nsplit_of_rank[r]
+ * splits as star_phase2_partial_ext writes them, [B, Hq, nsplit_of_rank[r],
+ * T, D] and [B, Hq, nsplit_of_rank[r], T]; the rest of the slot is ignored.
+ * nsplit_of_rank is a host array, 0 <= nsplit_of_rank[r] <= nsplit_stride,
+ * 1 <= nranks <= 64. Output and errors as star_lse_merge.
+ */
+star_status star_lse_merge_ranks(const float* part_o, const float* part_lse, int nranks,
+                                 const int* nsplit_of_rank, int nsplit_stride, void* o, float* lse,
+                                 int B, int T, int Hq, int D, void* cuda_stream);
 
 /*
  * star_phase2_decode_static — star_phase2_partial for decode steps

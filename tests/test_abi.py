@@ -101,12 +101,12 @@ def test_ext_workspace_sizes(lib):
 def _p1x(lib, **kw):
     a = dict(q=FAKE, k=FAKE, v=FAKE, o=FAKE, kc=FAKE, vc=FAKE, Lcap=64, lse=NULL, B=1, L=64,
              Hq=4, Hkv=2, D=64, b=16, src=FAKE, pos=FAKE, G=8, bounds=FAKE, xk=NULL, xv=NULL,
-             NX=0, theta=1e4, ws=FAKE, wsb=1 << 30)
+             NX=0, pos0=0, theta=1e4, ws=FAKE, wsb=1 << 30)
     a.update(kw)
     return lib.star_phase1_encode_ext(a["q"], a["k"], a["v"], a["o"], a["kc"], a["vc"], a["Lcap"],
                                       a["lse"], a["B"], a["L"], a["Hq"], a["Hkv"], a["D"], a["b"],
                                       a["src"], a["pos"], a["G"], a["bounds"], a["xk"], a["xv"],
-                                      a["NX"], a["theta"], a["ws"], a["wsb"], NULL)
+                                      a["NX"], a["pos0"], a["theta"], a["ws"], a["wsb"], NULL)
 
 
 @pytest.mark.parametrize("kw,status", [
@@ -121,6 +121,8 @@ def _p1x(lib, **kw):
     (dict(wsb=256 + 64 * 4 * 64 * 2), INVALID),  # room for Q only, not the table
     (dict(D=96), UNSUPPORTED),
     (dict(Lcap=63), INVALID),
+    (dict(pos0=-1), INVALID),
+    (dict(pos0=2**31 - 10), INVALID),      # ctx_pos0 + L past int32
 ])
 def test_phase1_ext_validation(lib, kw, status):
     assert _p1x(lib, **kw) == status
@@ -153,6 +155,46 @@ def test_phase2_validation(lib, kw, status):
     assert _p2(lib, **kw) == status
 
 
+def _p2x(lib, **kw):
+    a = dict(q=FAKE, k=FAKE, v=FAKE, T=1, kc=FAKE, vc=FAKE, Lcap=100, L=64, b=16, tail=0,
+             pos0=1000, qpos0=1064, with_tail=1, po=FAKE, pl=FAKE, B=1, Hq=4, Hkv=2, D=64,
+             theta=1e4, ws=FAKE, wsb=1 << 30)
+    a.update(kw)
+    ns = ctypes.c_int(-1)
+    return lib.star_phase2_partial_ext(a["q"], a["k"], a["v"], a["T"], a["kc"], a["vc"], a["Lcap"],
+                                       a["L"], a["b"], a["tail"], a["pos0"], a["qpos0"],
+                                       a["with_tail"], a["po"], a["pl"], ctypes.byref(ns), a["B"],
+                                       a["Hq"], a["Hkv"], a["D"], a["theta"], a["ws"], a["wsb"],
+                                       NULL)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(qpos0=1065), INVALID),                     # the tail must follow the cache
+    (dict(with_tail=2), INVALID),
+    (dict(with_tail=0, tail=3), INVALID),            # no tail split, no tail tokens
+    (dict(pos0=-1, qpos0=63), INVALID),
+    (dict(with_tail=0, qpos0=2**31 - 1), INVALID),   # q_pos0 + T past int32
+    (dict(k=NULL), INVALID),                         # the tail needs the new k/v
+    (dict(Lcap=64), INVALID),                        # no room for the new token
+    (dict(D=80), UNSUPPORTED),
+])
+def test_phase2_ext_validation(lib, kw, status):
+    assert _p2x(lib, **kw) == status
+    assert lib.star_last_error()
+
+
+def test_merge_ranks_validation(lib):
+    ns2 = (ctypes.c_int * 2)(3, 4)
+    ok_args = (FAKE, FAKE, 2, ns2, 4, FAKE, NULL, 1, 1, 4, 64, NULL)
+    assert lib.star_lse_merge_ranks(*((FAKE, FAKE, 0) + ok_args[3:])) == INVALID      # no ranks
+    assert lib.star_lse_merge_ranks(*((FAKE, FAKE, 65) + ok_args[3:])) == INVALID     # > 64 ranks
+    assert lib.star_lse_merge_ranks(*(ok_args[:4] + (3,) + ok_args[5:])) == INVALID   # 4 > stride 3
+    assert lib.star_lse_merge_ranks(*(ok_args[:3] + (None,) + ok_args[4:])) == INVALID
+    zero = (ctypes.c_int * 2)(0, 0)
+    assert lib.star_lse_merge_ranks(*(ok_args[:3] + (zero,) + ok_args[4:])) == INVALID  # nothing
+    assert lib.star_lse_merge_ranks(*(ok_args[:10] + (32, NULL))) == UNSUPPORTED
+
+
 def test_merge_and_rope_validation(lib):
     assert lib.star_lse_merge(FAKE, FAKE, 0, FAKE, NULL, 1, 1, 1, 64, NULL) == INVALID
     assert lib.star_lse_merge(FAKE, FAKE, 2, FAKE, NULL, 1, 1, 1, 32, NULL) == UNSUPPORTED
@@ -172,6 +214,8 @@ def test_valid_call_without_device_reports_cuda_error(lib):
     assert _p1(lib) in (CUDA, UNSUPPORTED)
     assert lib.star_last_error()
     assert _p1x(lib, G=0, src=NULL, pos=NULL, bounds=NULL) in (CUDA, UNSUPPORTED)
+    assert _p2x(lib) in (CUDA, UNSUPPORTED)
+    assert _p2x(lib, with_tail=0, k=NULL, v=NULL, qpos0=5000) in (CUDA, UNSUPPORTED)
 
 
 def test_python_binding_raises_on_missing_library(tmp_path):
