@@ -55,3 +55,40 @@ def make_new_tokens(B, T, Hq, Hkv, D, config_index, device="cpu"):
     k = make_tensor("k2", B, T, Hkv, D, config_index, device)
     v = make_tensor("v2", B, T, Hkv, D, config_index, device)
     return q, k, v
+
+
+# ---- decoder stack (random, untrained weights) --------------------------------
+STACK_ID = {"x": 0, "x2": 1, "gamma": 2, "wq": 3, "wk": 4, "wv": 5, "wo": 6}
+
+
+def stack_seed(config_index: int, layer: int, tensor_id: int) -> int:
+    return 100000 + 1000 * config_index + 10 * layer + tensor_id
+
+
+def make_hidden(B: int, S: int, dm: int, config_index: int, name: str = "x",
+                device="cpu") -> torch.Tensor:
+    """Hidden states [B, S, dm] bf16, N(0, 1), drawn on the CPU (the same
+    values on every device); name 'x' for the context, 'x2' for the
+    Phase-2 tokens."""
+    x = randn_bf16((B, S, dm), stack_seed(config_index, 999, STACK_ID[name]))
+    return x.to(device)
+
+
+def make_stack_weights(n_layers: int, dm: int, Hq: int, Hkv: int, D: int, config_index: int,
+                       device="cpu"):
+    """Per layer a dict: gamma [dm] ~ 1 + 0.1 N(0, 1); wq [Hq*D, dm], wk and
+    wv [Hkv*D, dm] ~ N(0, 1/dm); wo [dm, Hq*D] ~ N(0, 1/(Hq*D)). bf16, drawn
+    on the CPU."""
+    layers = []
+    for l in range(n_layers):
+        s = lambda name: stack_seed(config_index, l, STACK_ID[name])  # noqa: E731
+        g = torch.Generator().manual_seed(s("gamma"))
+        gamma = (1.0 + 0.1 * torch.randn(dm, generator=g)).to(torch.bfloat16)
+        layers.append({
+            "gamma": gamma.to(device),
+            "wq": randn_bf16((Hq * D, dm), s("wq"), scale=dm ** -0.5).to(device),
+            "wk": randn_bf16((Hkv * D, dm), s("wk"), scale=dm ** -0.5).to(device),
+            "wv": randn_bf16((Hkv * D, dm), s("wv"), scale=dm ** -0.5).to(device),
+            "wo": randn_bf16((dm, Hq * D), s("wo"), scale=(Hq * D) ** -0.5).to(device),
+        })
+    return layers

@@ -161,3 +161,34 @@ def gathered_prefix_literal(q, k, v, b, pk, pv, ppos, bounds, theta):
             o[own, h] = oo
             lse[h, own] = ll
     return o, lse
+
+
+def stack_literal(x0, layers, b, a, Hq, Hkv, D, theta, eps, rnd):
+    """Decoder stack with Star Phase 1 built literally: every block i >= 1
+    runs the whole stack on its own augmented sequence [c_1[:a] || c_i]
+    (anchor rows at positions 0..a-1, block rows at their own positions,
+    plain causal attention, the anchor recomputed in every block), block 0
+    on c_1 alone; the c_i rows are kept. x0 [L, dm] float64; layers: dicts
+    of float64 gamma/wq/wk/wv/wo; rnd: the rounding applied to every stored
+    intermediate (identity or bf16). Rotated q/k are rounded like the rest."""
+    L, dm = x0.shape
+    g = Hq // Hkv
+    out = np.empty_like(x0)
+    for i in range(-(-L // b)):
+        own = np.arange(i * b, min((i + 1) * b, L))
+        idx = own if (i == 0 or a == 0) else np.concatenate([np.arange(a), own])
+        X = x0[idx].copy()
+        S = idx.size
+        for ly in layers:
+            h = rnd(X / np.sqrt(np.mean(X * X, axis=-1, keepdims=True) + eps) * ly["gamma"])
+            q = rnd(h @ ly["wq"].T).reshape(S, Hq, D)
+            k = rnd(h @ ly["wk"].T).reshape(S, Hkv, D)
+            v = rnd(h @ ly["wv"].T).reshape(S, Hkv, D)
+            qr, kr = rnd(rope_complex(q, idx, theta)), rnd(rope_complex(k, idx, theta))
+            mask = np.tril(np.ones((S, S), dtype=bool))
+            o = np.empty((S, Hq, D))
+            for hq in range(Hq):
+                o[:, hq], _ = masked_attention(qr[:, hq], kr[:, hq // g], v[:, hq // g], mask)
+            X = rnd(X + rnd(o.reshape(S, Hq * D)) @ ly["wo"].T)
+        out[own] = X[S - own.size:]
+    return out
