@@ -189,6 +189,6 @@ def stack_literal(x0, layers, b, a, Hq, Hkv, D, theta, eps, rnd):
             o = np.empty((S, Hq, D))
             for hq in range(Hq):
                 o[:, hq], _ = masked_attention(qr[:, hq], kr[:, hq // g], v[:, hq // g], mask)
-            X = rnd(X + rnd(o.reshape(S, Hq * D)) @ ly["wo"].T)
+            X = rnd(X + rnd(rnd(o.reshape(S, Hq * D)) @ ly["wo"].T))
         out[own] = X[S - own.size:]
     return out

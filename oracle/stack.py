@@ -5,8 +5,9 @@ Star Attention replaces only attention and needs no retraining [pith
 2WVXFXZ2, the paper's abstract]. A layer here is an attention block:
     h = RMSNorm(x) * gamma;  q, k, v = h Wq^T, h Wk^T, h Wv^T;
     o = Star Phase 1 (or, for new tokens, global attention);  x = x + o Wo^T
-with every stored intermediate (h, q, k, v, o, x) rounded to bf16, as the
-GPU path stores them. The attention is the fp64 oracle of this package
+with every stored intermediate (h, q, k, v, o, the projection o Wo^T and x)
+rounded to bf16, as the GPU path stores them: the residual add rounds the
+bf16 projection output plus x once more. The attention is the fp64 oracle of this package
 (phase1_full / global_rows), so in layer l every block's anchor is the
 layer-l hidden state of rows 0..a-1 of the whole sequence — block 1's, since
 the anchor is a causal prefix of every augmented block [pith 2WVXFXZ2, "What
@@ -50,7 +51,7 @@ def stack_encode(x0, layers, block_len, anchor_len, Hq, Hkv, D, theta, eps=1e-5)
         v = rnd(h @ _f64(ly["wv"]).T).reshape(B, L, Hkv, D)
         o, _ = orc.phase1_full(_bf16(q), _bf16(k), _bf16(v), block_len, anchor_len, theta)
         o = rnd(o).reshape(B, L, Hq * D)
-        x = rnd(x + o @ _f64(ly["wo"]).T)
+        x = rnd(x + rnd(o @ _f64(ly["wo"]).T))
         kv.append((_bf16(k), _bf16(v)))
     return x, kv
 
@@ -76,5 +77,5 @@ def stack_step(x_new, layers, ctx_kv, new_kv, tail_len, Hq, Hkv, D, theta, eps=1
         o, _ = orc.global_rows(q, kc, vc, kt, vt, tail_len, theta, bb.ravel(), hh.ravel(),
                                tt.ravel())
         o = rnd(o.reshape(B, Hq, T, D).transpose(0, 2, 1, 3)).reshape(B, T, Hq * D)
-        x = rnd(x + o @ _f64(ly["wo"]).T)
+        x = rnd(x + rnd(o @ _f64(ly["wo"]).T))
     return x
