@@ -10,6 +10,11 @@ merge). Inputs are resident in HBM when the timed region starts.
 One JSON line on stdout (rank 0). With N > 1 (torchrun, one rank per GPU)
 each rank runs its own independent sequences (weak scaling, no data-path
 collective); the time is the max over ranks.
+
+--mode sharded spreads ONE sequence's blocks over the N ranks instead (the
+pages' multi-host form: Phase 1 per shard, Phase 2 with a query broadcast, an
+all-gather of partials and the merge over NCCL; strong scaling), launched
+eagerly. With N = 1 it runs the same code on a one-rank process group.
 """
 import argparse
 import json
@@ -341,6 +346,37 @@ def run_star(args, w, rank, world, local_rank):
         pul_ms = max_over_ranks([s3.elapsed_time(e3) / args.steps], dev, world)[0]
         pulsar = (pul_ms, pfx.prefix_pairs(w.L, w.block_len, bounds), int(src.size))
 
+    # ---- a decoder stack around Star attention (a side measurement outside
+    # the step): RMSNorm, Q/K/V/O projections (cuBLASLt) and Phase 1 per layer
+    stack_res = None
+    if args.stack_layers > 0:
+        from block_sparse_long_rope_b200.stack import StarStack
+        dm = w.Hq * w.D
+        wts = inputs.make_stack_weights(args.stack_layers, dm, w.Hq, w.Hkv, w.D, w.index,
+                                        device=dev)
+        stk = StarStack(w, dm, wts, device=dev)
+        x0 = inputs.make_hidden(w.B, w.L, dm, w.index, device=dev)
+        xs = torch.empty_like(x0)
+        for _ in range(args.warmup):
+            xs.copy_(x0)
+            stk.encode(xs)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        sev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        for i in range(args.steps):
+            xs.copy_(x0)  # a fresh residual stream each pass (outside the events)
+            sev[i][0].record(stream)
+            stk.encode(xs)
+            sev[i][1].record(stream)
+        torch.cuda.synchronize()
+        for ly in stk.layers:
+            star.star_device_status(ly.buf.ws1)
+        st_ms = max_over_ranks([sum(e[0].elapsed_time(e[1]) for e in sev) / args.steps], dev,
+                               world)[0]
+        stack_res = (st_ms, stk.flops_encode(), dm)
+        del stk, wts, x0, xs
+
     if rank != 0:
         return None
 
@@ -398,6 +434,15 @@ def run_star(args, w, rank, world, local_rank):
                         "chunks (12.5% of a block, seeded draw standing in for Max-IDF); block i "
                         "sees sink + summaries of blocks < i at original positions; "
                         "gather/rope + rope + attention kernels"}}),
+            **({} if stack_res is None else {"stack_encode": {
+                "layers": args.stack_layers, "d_model": stack_res[2],
+                "ms": round(stack_res[0], 4),
+                "ctx_tok_s": round(w.B * w.L / (stack_res[0] / 1e3), 1),
+                "tflops": round(stack_res[1] / (stack_res[0] / 1e3) / 1e12, 2),
+                "frac_bf16_peak": round(stack_res[1] / (stack_res[0] / 1e3) / 1e12 / bf16_peak, 4),
+                "note": "per layer: star_rmsnorm, Q/K/V projections and the O projection with "
+                        "the residual (cuBLASLt GEMMs), star_phase1_encode; random weights; "
+                        "FLOPs = projections + Phase-1 unmasked attention"}}),
             "phase2_query_chunk": {"ms": round(chunk_s * 1e3, 4), "tokens": w.Tq,
                                    "tflops": round(4.0 * w.D * w.Hq * w.B * w.Tq * w.L / chunk_s / 1e12, 2)},
             "phase2_decode": {"ms": round(dec_s * 1e3, 4), "tok_s": round(dec_tok_s, 1),
@@ -419,6 +464,159 @@ def run_star(args, w, rank, world, local_rank):
         "e2e": {"value": round(job_value(w.B * w.L, world, e2e_ms / K), 1), "unit": "tok/s",
                 "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
         "gpu_launches": launches * K,
+        "clocks": clocks,
+    }
+    if args.cpu_baseline:
+        est_step, sample, spent = oracle_sample(w, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(w.B * w.L / est_step, 3), "unit": "tok/s",
+                                "cores": omp_threads(), "kind": "oracle", "sample": sample,
+                                "seconds_spent": round(spent, 2), "extrapolated": True}
+    return line
+
+
+def run_sharded(args, w, rank, world, local_rank):
+    """One sequence over the ranks (block_sparse_long_rope_b200.sharded)."""
+    import torch
+    import torch.distributed as dist
+
+    from block_sparse_long_rope_b200 import inputs, sharded, star
+    from block_sparse_long_rope_b200.pipeline import phase2_calls
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks, peak_src = load_peaks()
+    plan = sharded.shard_plan(w.L, w.block_len, world)
+    sh = plan[rank]
+    with torch.no_grad():
+        q, k, v = inputs.make_context(w.B, w.L, w.Hq, w.Hkv, w.D, w.index, device=dev)
+        rows = slice(sh.row0, sh.row0 + sh.rows)
+        ctx = [t[:, rows].contiguous() for t in (q, k, v)]
+        anchor = [t[:, :w.anchor_len].contiguous() for t in (k, v)]
+        del q, k, v
+        new = inputs.make_new_tokens(w.B, w.Tq + w.Tdec, w.Hq, w.Hkv, w.D, w.index, device=dev)
+    calls = phase2_calls(w, *new)
+    layer = sharded.ShardedStarLayer(w, plan, rank, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        layer.encode(*ctx, anchor_k=anchor[0], anchor_v=anchor[1])
+        if ev is not None:
+            ev[1].record(stream)
+        out = None
+        for (q2, k2, v2, tail) in calls:
+            out = layer.attend(q2, k2, v2, tail)
+        if ev is not None:
+            ev[2].record(stream)
+        return out
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    star.star_device_status(layer.ws1)
+    star.star_device_status(layer.ws2)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(args.steps):
+        step(evs[i])
+    end.record(stream)
+    torch.cuda.synchronize()
+    dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    p1_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    p2_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    elapsed_ms, p1_ms, p2_ms = max_over_ranks([start.elapsed_time(end), p1_ms, p2_ms], dev, world)
+
+    # end to end: this rank's shard and the anchor rows from pinned host memory
+    host_ctx = [t.cpu().pin_memory() for t in ctx + anchor]
+    host_calls = [tuple(x.cpu().pin_memory() for x in c[:3]) + (c[3],) for c in calls]
+    dev_ctx = [torch.empty_like(t) for t in ctx + anchor]
+    dev_calls = [tuple(torch.empty_like(x) for x in c[:3]) + (c[3],) for c in calls]
+    host_o = torch.empty(layer.o.shape, dtype=torch.bfloat16).pin_memory()
+    host_dec = torch.empty((w.B, 1, w.Hq, w.D), dtype=torch.bfloat16).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_ctx) + \
+        sum(x.numel() * x.element_size() for c in host_calls for x in c[:3])
+    d2h = host_o.numel() * 2 + host_dec.numel() * 2
+
+    def e2e_step():
+        for d, h in zip(dev_ctx, host_ctx):
+            d.copy_(h, non_blocking=True)
+        for dc, hc in zip(dev_calls, host_calls):
+            for d, h in zip(dc[:3], hc[:3]):
+                d.copy_(h, non_blocking=True)
+        layer.encode(*dev_ctx[:3], anchor_k=dev_ctx[3], anchor_v=dev_ctx[4])
+        out = None
+        for (q2, k2, v2, tail) in dev_calls:
+            out = layer.attend(q2, k2, v2, tail)
+        host_o.copy_(layer.o, non_blocking=True)
+        host_dec.copy_(out[0], non_blocking=True)
+
+    for _ in range(max(1, args.warmup // 2)):
+        e2e_step()
+    torch.cuda.synchronize()
+    dist.barrier()
+    s2 = torch.cuda.Event(enable_timing=True)
+    e2 = torch.cuda.Event(enable_timing=True)
+    s2.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e2.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks([s2.elapsed_time(e2)], dev, world)[0]
+    if rank != 0:
+        return None
+
+    K = args.steps
+    ms_step = elapsed_ms / K
+    p1_s = p1_ms / K / 1e3
+    p1_tflops_gpu = w.phase1_flops() / p1_s / 1e12 / world
+    bf16_peak = float(peaks["bf16_tflops"])
+    p1_launches = 2 if sh.first_block == 0 else 3
+    line = {
+        "metric": METRIC,
+        "value": round(w.B * w.L / (ms_step / 1e3), 1),
+        "unit": "tok/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True,
+        "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic N(0,1) bf16 Q/K/V (seeded), one sequence sharded by blocks",
+        "config": {
+            "workload": w.name, "B": w.B, "L": w.L, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
+            "block_len": w.block_len, "anchor_len": w.anchor_len, "theta": w.theta,
+            "Tq": w.Tq, "Tdec": w.Tdec, "global_batch": w.B, "seq_len": w.L,
+            "parallelism": f"sequence-sharded{world}", "launch": "eager",
+            "l2": "step inputs exceed the 126 MB L2 at 16K and up; no flush",
+        },
+        "phases": {
+            "phase1": {"ms": round(p1_s * 1e3, 4),
+                       "unmasked_tflops_per_gpu": round(p1_tflops_gpu, 2),
+                       "note": "slowest rank's Phase 1 (star_phase1_encode or _ext on its shard)"},
+            "phase2": {"ms": round(p2_ms / K, 4),
+                       "note": "query chunk + decode steps: broadcast, partials, all-gather, merge"},
+        },
+        "roofline": {"bound": "tensor", "kernel": "phase1 (per-shard encode)",
+                     "achieved": round(p1_tflops_gpu, 2), "peak": bf16_peak, "unit": "TFLOP/s",
+                     "frac": round(p1_tflops_gpu / bf16_peak, 4),
+                     "peak_source": f"{peak_src} bf16_tflops (burst)",
+                     "algorithmic": "whole-sequence Phase-1 unmasked FLOPs / slowest rank / N",
+                     "traffic": None},
+        "e2e": {"value": round(w.B * w.L / (e2e_ms / K / 1e3), 1), "unit": "tok/s",
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+        "gpu_launches": (p1_launches + 3 + 2 * w.Tdec) * K,
         "clocks": clocks,
     }
     if args.cpu_baseline:
@@ -460,6 +658,14 @@ def run_reference(args, w, rank):
     }
 
 
+def _free_port():
+    import socket
+
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -472,6 +678,11 @@ def main():
                     help="launch every call directly instead of replaying CUDA graphs")
     ap.add_argument("--no-pulsar", dest="pulsar", action="store_false",
                     help="skip the side measurement of Phase 1 with Pulsar's prefix layout")
+    ap.add_argument("--stack-layers", type=int, default=2,
+                    help="layers of the side measurement of a decoder stack (0 skips it)")
+    ap.add_argument("--mode", default="replicas", choices=["replicas", "sharded"],
+                    help="replicas: independent sequences per rank; sharded: one sequence's "
+                         "blocks spread over the ranks")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=8.0)
     args = ap.parse_args()
@@ -488,19 +699,26 @@ def main():
         if line is not None:
             print(json.dumps(line), flush=True)
         return
-    if world > 1:
+    use_pg = world > 1 or args.mode == "sharded"
+    if use_pg:
         import datetime
 
         import torch
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
-        dist.init_process_group(backend="nccl", timeout=datetime.timedelta(seconds=120))
+        if world == 1:
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            os.environ.setdefault("MASTER_PORT", str(_free_port()))
+        dist.init_process_group(backend="nccl", rank=rank, world_size=world,
+                                timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
     try:
-        line = run_star(args, w, rank, world, local_rank)
+        run = run_sharded if args.mode == "sharded" else run_star
+        line = run(args, w, rank, world, local_rank)
         if rank == 0 and line is not None:
             print(json.dumps(line), flush=True)
     finally:
-        if world > 1:
+        if use_pg:
             import torch.distributed as dist
             dist.destroy_process_group()
 

@@ -35,6 +35,8 @@ EXPORTS = (
     "star_phase2_decode_static",
     "star_phase2_attend",
     "star_lse_merge",
+    "star_rmsnorm",
+    "star_linear",
     "star_device_status",
     "star_debug_index",
     "star_debug_wait_probe",
@@ -92,6 +94,10 @@ def load(path: str = LIB_PATH):
                                                 _P, _P, _IP, _I, _I, _I, _I, _D, _P, _SZ, _P]
         lib.star_lse_merge_ranks.restype = _I
         lib.star_lse_merge_ranks.argtypes = [_P, _P, _I, _IP, _I, _P, _P, _I, _I, _I, _I, _P]
+        lib.star_rmsnorm.restype = _I
+        lib.star_rmsnorm.argtypes = [_P, _P, _P, _I, _I, ctypes.c_float, _P]
+        lib.star_linear.restype = _I
+        lib.star_linear.argtypes = [_P, _P, _P, _I, _I, _I, _I, _P, _SZ, _P]
         lib.star_phase2_workspace_bytes.restype = _SZ
         lib.star_phase2_workspace_bytes.argtypes = [_I, _I, _I, _I, _I, _I, _I]
         lib.star_phase2_partial.restype = _I

@@ -13,7 +13,8 @@ INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libstar.so")
 OBJ_DIR = os.path.join(HERE, "_build")
 
-SOURCES = ["api.cu", "rope.cu", "lse_merge.cu", "phase2_decode.cu", "phase1_sm100.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "rope.cu", "lse_merge.cu", "phase2_decode.cu", "phase1_sm100.cu", "noalloc.cu",
+           "stack.cu"]
 HEADERS = ["star_common.cuh", "star_index.cuh", "star_kernels.cuh", "rope_math.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
@@ -43,7 +44,7 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
             subprocess.check_call(cmd)
     if force or _stale(LIB, objs):
         tmp = LIB + f".tmp{os.getpid()}"
-        cmd = [NVCC] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", tmp] + objs
+        cmd = [NVCC] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", tmp] + objs + ["-lcublasLt"]
         subprocess.check_call(cmd)
         os.replace(tmp, LIB)
     return LIB

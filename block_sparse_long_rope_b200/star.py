@@ -241,6 +241,36 @@ def star_lse_merge_ranks(part_o, part_lse, nsplit_of_rank, slots, o, lse=None, s
     return o
 
 
+def star_rmsnorm(x, gamma, y, eps=1e-5, stream=None):
+    """y = x / rms(x) * gamma over the last dim (bf16 [..., dm])."""
+    for t, n in ((x, "x"), (gamma, "gamma"), (y, "y")):
+        _bf16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    dm = x.shape[-1]
+    lib = _abi.load()
+    _abi.check(lib.star_rmsnorm(_ptr(x), _ptr(gamma), _ptr(y), x.numel() // dm, dm, float(eps),
+                                _stream(stream)))
+    return y
+
+
+def star_linear(x, w, y, accumulate=False, workspace=None, stream=None):
+    """y[M, N] = x[M, K] w[N, K]^T (+ y when accumulate), bf16 row-major."""
+    for t, n in ((x, "x"), (w, "w"), (y, "y")):
+        _bf16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    N, K = w.shape
+    M = x.numel() // K
+    if y.numel() != M * N:
+        raise ValueError("y must hold M x N elements")
+    wsb = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    lib = _abi.load()
+    _abi.check(lib.star_linear(_ptr(x), _ptr(w), _ptr(y), M, N, K, 1 if accumulate else 0,
+                               _ptr(workspace), wsb, _stream(stream)))
+    return y
+
+
 def star_device_status(workspace, stream=None):
     """Synchronise, read and clear the device status word; raises on a device error."""
     lib = _abi.load()

@@ -291,6 +291,33 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
                                       int D, double theta, void* cuda_stream);
 
 /*
+ * Layers around Star attention in a decoder stack. Star Attention replaces
+ * only attention and needs no retraining [pith 2WVXFXZ2, the paper's
+ * abstract]; in a stack every layer encodes its own anchor, whose hidden
+ * state is block 1's at that layer because the anchor is a causal prefix of
+ * every augmented block [pith 2WVXFXZ2, "What carries the argument"]. These
+ * two calls supply the row-wise parts of an attention block:
+ *
+ * star_rmsnorm — y[r, :] = x[r, :] / sqrt(mean(x[r, :]^2) + eps) * gamma,
+ *   x, y bf16 [rows, dm] (row-major, may alias), gamma bf16 [dm]; fp32
+ *   arithmetic, one rounding to bf16. dm a multiple of 8, pointers 16-byte
+ *   aligned. STAR_ERR_INVALID_ARG otherwise; STAR_ERR_CUDA if the launch fails.
+ *
+ * star_linear — y[M, N] = x[M, K] * w[N, K]^T (+ y[M, N] if accumulate = 1,
+ *   the residual add), bf16 row-major operands, fp32 accumulation, one
+ *   rounding to bf16. A plain GEMM: it runs in cuBLASLt. N and K multiples of
+ *   8, pointers 16-byte aligned; workspace (optional, caller-owned, 256-byte
+ *   aligned) is cuBLASLt's scratch. The library keeps one cuBLASLt handle and
+ *   a cache of chosen algorithms per (device, shape); it allocates no device
+ *   memory. STAR_ERR_INVALID_ARG for bad shapes or pointers, STAR_ERR_CUDA for
+ *   a cuBLASLt failure (message names the step).
+ */
+star_status star_rmsnorm(const void* x, const void* gamma, void* y, int rows, int dm, float eps,
+                         void* cuda_stream);
+star_status star_linear(const void* x, const void* w, void* y, int M, int N, int K, int accumulate,
+                        void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
  * star_device_status — synchronises `cuda_stream`, then reads and clears the
  * status word at the start of `workspace` (a workspace passed to
  * star_phase1_encode or star_phase2_partial). Returns STAR_OK,

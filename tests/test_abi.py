@@ -195,6 +195,24 @@ def test_merge_ranks_validation(lib):
     assert lib.star_lse_merge_ranks(*(ok_args[:10] + (32, NULL))) == UNSUPPORTED
 
 
+def test_stack_calls_validation(lib):
+    # RMSNorm: dm a multiple of 8, aligned non-NULL pointers, eps >= 0
+    assert lib.star_rmsnorm(FAKE, FAKE, FAKE, 4, 12, 1e-5, NULL) == INVALID
+    assert lib.star_rmsnorm(FAKE, FAKE, FAKE, -1, 64, 1e-5, NULL) == INVALID
+    assert lib.star_rmsnorm(FAKE, NULL, FAKE, 4, 64, 1e-5, NULL) == INVALID
+    assert lib.star_rmsnorm(FAKE, FAKE, ODD, 4, 64, 1e-5, NULL) == INVALID
+    assert lib.star_rmsnorm(FAKE, FAKE, FAKE, 4, 64, -1.0, NULL) == INVALID
+    # linear: N, K multiples of 8, accumulate 0/1, aligned workspace
+    assert lib.star_linear(FAKE, FAKE, FAKE, 4, 12, 64, 0, NULL, 0, NULL) == INVALID
+    assert lib.star_linear(FAKE, FAKE, FAKE, 4, 64, 60, 0, NULL, 0, NULL) == INVALID
+    assert lib.star_linear(FAKE, FAKE, FAKE, 0, 64, 64, 0, NULL, 0, NULL) == INVALID
+    assert lib.star_linear(FAKE, FAKE, FAKE, 4, 64, 64, 2, NULL, 0, NULL) == INVALID
+    assert lib.star_linear(NULL, FAKE, FAKE, 4, 64, 64, 0, NULL, 0, NULL) == INVALID
+    assert lib.star_linear(FAKE, FAKE, FAKE, 4, 64, 64, 0, NULL, 1024, NULL) == INVALID
+    assert lib.star_linear(FAKE, FAKE, FAKE, 4, 64, 64, 0, ODD, 1024, NULL) == INVALID
+    assert lib.star_last_error()
+
+
 def test_merge_and_rope_validation(lib):
     assert lib.star_lse_merge(FAKE, FAKE, 0, FAKE, NULL, 1, 1, 1, 64, NULL) == INVALID
     assert lib.star_lse_merge(FAKE, FAKE, 2, FAKE, NULL, 1, 1, 1, 32, NULL) == UNSUPPORTED
