@@ -174,6 +174,23 @@ int decode_chunk(int B, int Hkv, int L, int b, int n, int nsplit, int tail_plus_
   long long chunk_tiles = room > 0 ? (total_tiles + room - 1) / room : max_split_tiles;
   chunk_tiles = std::max<long long>(chunk_tiles, ceil_div(max_split_tiles, star::kMaxChunksPerSplit));
   chunk_tiles = std::max<long long>(1, std::min<long long>(chunk_tiles, max_split_tiles));
+  // equal units within a full block: the same number of units, none ragged
+  // (64 tiles in chunks of 9 would leave a 1-tile unit; 8 x 8 balances them).
+  // Kept only if the split limit holds and the unit count stays within one
+  // wave (or the count before), which the scratch size assumes.
+  const long long block_tiles = ceil_div(imin(b, L), tile);
+  const long long last_tiles = ceil_div(L - (n - 1) * b, tile);
+  const long long tail_tiles = ceil_div(tail_plus_T, tile);
+  auto units_for = [&](long long ct) {
+    return (long long)B * Hkv *
+           ((n - 1) * ((block_tiles + ct - 1) / ct) + (last_tiles + ct - 1) / ct +
+            (tail_tiles + ct - 1) / ct);
+  };
+  const long long per_block = (block_tiles + chunk_tiles - 1) / chunk_tiles;
+  const long long even = std::max<long long>(
+      (block_tiles + per_block - 1) / per_block,
+      ceil_div(max_split_tiles, star::kMaxChunksPerSplit));
+  if (units_for(even) <= std::max(units_for(chunk_tiles), ctas)) chunk_tiles = even;
   return static_cast<int>(chunk_tiles) * tile;
 }
 
@@ -318,8 +335,7 @@ star_status phase1_run(const void* q, const void* k, const void* v, void* o, voi
   __nv_bfloat16* pk_buf = reinterpret_cast<__nv_bfloat16*>(ws + star::kStatusBytes + qrot_bytes);
   __nv_bfloat16* pv_buf =
       reinterpret_cast<__nv_bfloat16*>(ws + star::kStatusBytes + qrot_bytes + tbl_bytes);
-  cudaError_t e = cudaMemsetAsync(ws, 0, star::kStatusBytes, st);
-  if (e != cudaSuccess) return cuda_fail(e, "status reset");
+  cudaError_t e;
 
   // RoPE: Q -> workspace (token-major), K -> k_cache (head-major, rotated),
   // V -> v_cache (head-major copy). Token t sits at position t.
@@ -437,10 +453,11 @@ star_status star_phase1_encode_ext(const void* q, const void* k, const void* v, 
 size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lcap, int block_len) {
   if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || D < 1 || Lcap < 1 || block_len < 1 || Hq % Hkv)
     return star::kStatusBytes;
-  if (use_decode_path(T, Hq, Hkv))
-    return decode_header_bytes(B, Hkv, Lcap, block_len) + align_up((size_t)B * T * Hq * D * 2) +
-           decode_scratch_bytes(B, Hkv, D, Lcap, block_len);
-  return star::kStatusBytes + align_up((size_t)B * T * Hq * D * 2);
+  // every Phase-2 call keeps the decode header (status block and counters)
+  // in front, so query-chunk and decode calls can share one workspace
+  const size_t head = decode_header_bytes(B, Hkv, Lcap, block_len) + align_up((size_t)B * T * Hq * D * 2);
+  if (use_decode_path(T, Hq, Hkv)) return head + decode_scratch_bytes(B, Hkv, D, Lcap, block_len);
+  return head;
 }
 
 }  // extern "C"
@@ -496,12 +513,14 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   const bool decode = use_decode_path(T, Hq, Hkv);
-  // zeroed header (status word; split counters on the decode path), then the rotated q
-  const size_t header = decode ? decode_header_bytes(B, Hkv, Lcap, block_len) : star::kStatusBytes;
+  // header (status block, then the decode path's split and head counters,
+  // which the decode kernel returns to zero; reserved on every Phase-2 path
+  // so a workspace can serve query chunks and decode steps alike), then the
+  // rotated q
+  const size_t header = decode_header_bytes(B, Hkv, Lcap, block_len);
   __nv_bfloat16* qrot = reinterpret_cast<__nv_bfloat16*>(ws + header);
   const size_t qrot_bytes = align_up((size_t)B * T * Hq * D * 2);
-  cudaError_t e = cudaMemsetAsync(ws, 0, header, st);
-  if (e != cudaSuccess) return cuda_fail(e, "status reset");
+  cudaError_t e;
 
   // RoPE of the new tokens at positions q_pos0 + t; with the tail, K/V
   // appended to cache rows L + tail_len + t. The decode kernel does both itself.
@@ -577,6 +596,7 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
     dp.part_o = part_o;
     dp.part_lse = part_lse;
     dp.status = reinterpret_cast<int*>(ws);
+    dp.header_bytes = static_cast<int>(header);
     dp.scale_ln = (float)(1.0 / sqrt((double)D));
     dp.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
     e = star::launch_decode(dp, D, st);
@@ -722,11 +742,18 @@ star_status star_device_status(void* workspace, void* cuda_stream) {
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   cudaError_t e = cudaStreamSynchronize(st);
   if (e != cudaSuccess) return cuda_fail(e, "stream synchronize");
-  int word = 0;
-  e = cudaMemcpy(&word, workspace, sizeof word, cudaMemcpyDeviceToHost);
+  // word 0: the status bits (sticky until read here); word 1: the size of the
+  // header the last decode call counted in, cleared with the status after an
+  // error (an aborted call may leave its counters non-zero)
+  int words[2] = {0, 0};
+  e = cudaMemcpy(words, workspace, sizeof words, cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(e, "status read");
-  e = cudaMemset(workspace, 0, sizeof word);
-  if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  const int word = words[0];
+  if (word != 0) {
+    const size_t clear = std::max<size_t>(sizeof word, static_cast<size_t>(std::max(words[1], 0)));
+    e = cudaMemset(workspace, 0, clear);
+    if (e != cudaSuccess) return cuda_fail(e, "status clear");
+  }
   if (word & star::kDevTimeout)
     return fail(STAR_ERR_DEVICE_TIMEOUT, "a kernel's bounded wait gave up (status 0x%x)", word);
   if (word & star::kDevBounds)

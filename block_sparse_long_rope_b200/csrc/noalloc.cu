@@ -239,6 +239,7 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
   dp.part_o = part_o;
   dp.part_lse = part_lse;
   dp.status = reinterpret_cast<int*>(ws);
+  dp.header_bytes = static_cast<int>(zero_bytes);
   dp.counters = reinterpret_cast<int*>(ws + star::kStatusBytes);
   dp.scale_ln = (float)(1.0 / sqrt((double)D));
   dp.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));

@@ -35,6 +35,7 @@ namespace {
 
 constexpr int kDecStages = 3;
 constexpr int kDecThreads = 160;  // 4 consumer warps + 1 producer warp
+constexpr int kTabPairs = 256;    // (token, frequency) cos/sin pairs per table round
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {
@@ -132,139 +133,93 @@ __device__ __forceinline__ void split_chunks(const DecodeParams& p, int split, i
   }
 }
 
+// Weighted LSE combine of `count` partials (lse l_j, normalised rows o_j) of
+// one row, four columns at a time: o = sum_j w_j o_j / sum_j w_j, lse = M +
+// log sum_j w_j with w_j = e^(l_j - M), M = max_j l_j. The partials are read
+// in batches of kBatch with all loads of a batch issued together, the max
+// taken in registers (one round trip per batch, no shared memory); a later
+// batch with a larger max rescales the running sums.
+template <int kBatch, typename LseAt, typename OAt>
+__device__ __forceinline__ float4 lse_combine(int count, LseAt lse_at, OAt o_at, float* lse_out) {
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  float z = 0.f, M = -INFINITY;
+  for (int c0 = 0; c0 < count; c0 += kBatch) {
+    float l[kBatch];
+    float4 v[kBatch];
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const bool in = c0 + j < count;
+      l[j] = in ? lse_at(c0 + j) : -INFINITY;
+      v[j] = in ? o_at(c0 + j) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    float mb = M;
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) mb = fmaxf(mb, l[j]);
+    if (mb == -INFINITY) continue;
+    if (mb > M) {
+      const float a = (M == -INFINITY) ? 0.f : expf(M - mb);
+      acc = make_float4(acc.x * a, acc.y * a, acc.z * a, acc.w * a);
+      z *= a;
+      M = mb;
+    }
+#pragma unroll
+    for (int j = 0; j < kBatch; ++j) {
+      const float w = (l[j] == -INFINITY) ? 0.f : expf(l[j] - M);
+      acc = make_float4(acc.x + w * v[j].x, acc.y + w * v[j].y, acc.z + w * v[j].z,
+                        acc.w + w * v[j].w);
+      z += w;
+    }
+  }
+  const float inv = (z > 0.f) ? 1.f / z : 0.f;
+  *lse_out = (z > 0.f) ? M + logf(z) : -INFINITY;
+  return make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+}
+
 // Reduce the chunk partials of one split (fixed order) into part_o /
 // part_lse. Run by the consumer warps of the CTA that finished the split's
-// last chunk; `sw` is free shared memory of kDecRows * (kMaxChunksPerSplit + 2)
-// floats.
+// last chunk; each thread owns (row, 4 columns) items.
 template <int D>
-__device__ void reduce_split(const DecodeParams& p, int bh, int split, float* sw) {
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  constexpr int kC = kMaxChunksPerSplit;
-  const int nsplit = p.nsplit;
+__device__ void reduce_split(const DecodeParams& p, int bh, int split) {
   int first, count;
   split_chunks(p, split, &first, &count);
   const size_t cbase = static_cast<size_t>(bh) * p.chunks_per_head + first;
-  float* wgt = sw;                // [R][kC] weights exp(lse_c - M)
-  float* rowz = sw + kDecRows * kC;  // [R] sum of weights
-  float* rowm = rowz + kDecRows;  // [R] max statistic
-  for (int rho = warp; rho < p.R; rho += kConsumers / 32) {
-    float M = -INFINITY;
-    for (int c = lane; c < count; c += 32) M = fmaxf(M, p.ws_lse[(cbase + c) * kDecRows + rho]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float z = 0.f;
-    for (int c = lane; c < count; c += 32) {
-      const float l = p.ws_lse[(cbase + c) * kDecRows + rho];
-      const float wv = (M == -INFINITY || l == -INFINITY) ? 0.f : expf(l - M);
-      wgt[rho * kC + c] = wv;
-      z += wv;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    if (lane == 0) {
-      rowz[rho] = z;
-      rowm[rho] = M;
-    }
-  }
-  consumer_sync();
-  // 4 columns per thread; the chunk loads of a group of 16 are all issued
-  // before any is used (the reduction is latency-bound)
-  for (int idx = tid; idx < p.R * (D / 4); idx += kConsumers) {
+  const int b = bh / p.Hkv;
+  for (int idx = threadIdx.x; idx < p.R * (D / 4); idx += kConsumers) {
     const int rho = idx / (D / 4), d4 = idx % (D / 4);
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int c0 = 0; c0 < count; c0 += 16) {
-      float4 v[16];
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        v[j] = (c0 + j < count)
-                   ? reinterpret_cast<const float4*>(p.ws_o + ((cbase + c0 + j) * kDecRows + rho) * D)[d4]
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float wv = (c0 + j < count) ? wgt[rho * kC + c0 + j] : 0.f;
-        acc.x += wv * v[j].x;
-        acc.y += wv * v[j].y;
-        acc.z += wv * v[j].z;
-        acc.w += wv * v[j].w;
-      }
-    }
-    const float z = rowz[rho];
-    const float inv = (z > 0.f) ? 1.f / z : 0.f;
+    float lse;
+    const float4 o = lse_combine<16>(
+        count, [&](int c) { return p.ws_lse[(cbase + c) * kDecRows + rho]; },
+        [&](int c) { return reinterpret_cast<const float4*>(p.ws_o + ((cbase + c) * kDecRows + rho) * D)[d4]; },
+        &lse);
     const int t = rho / p.g, h = (bh % p.Hkv) * p.g + rho % p.g;
-    const int b = bh / p.Hkv;
-    const size_t row = ((static_cast<size_t>(b) * p.Hq + h) * nsplit + split) * p.T + t;
-    reinterpret_cast<float4*>(p.part_o + row * D)[d4] =
-        make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
-    if (d4 == 0) p.part_lse[row] = (z > 0.f) ? rowm[rho] + logf(z) : -INFINITY;
+    const size_t row = ((static_cast<size_t>(b) * p.Hq + h) * p.nsplit + split) * p.T + t;
+    reinterpret_cast<float4*>(p.part_o + row * D)[d4] = o;
+    if (d4 == 0) p.part_lse[row] = lse;
   }
 }
 
-// Exact LSE merge of the n+1 split partials of one (batch, KV head) into
+// Exact LSE merge of the split partials of one (batch, KV head) into
 // o_merged / lse_merged: m = max lse_s, w_s = exp(lse_s - m),
-// o = sum w_s o_s / sum w_s, lse = m + log(sum w_s). Consumer warps only.
+// o = sum w_s o_s / sum w_s, lse = m + log(sum w_s) [pith 2WVXFXZ2, minor
+// comment on Algorithm 2]. Consumer warps only.
 template <int D>
-__device__ void merge_head(const DecodeParams& p, int bh, float* sw) {
-  const int tid = threadIdx.x, warp = tid / 32, lane = tid % 32;
-  const int nsplit = p.nsplit;
+__device__ void merge_head(const DecodeParams& p, int bh) {
   const int b = bh / p.Hkv, kvh = bh % p.Hkv;
-  float* rowm = sw;             // [R]
-  float* rowz = sw + kDecRows;  // [R]
-  auto prow = [&](int rho, int sp) {  // row index into part_o / part_lse
-    const int t = rho / p.g, h = kvh * p.g + rho % p.g;
-    return ((static_cast<size_t>(b) * p.Hq + h) * nsplit + sp) * p.T + t;
-  };
-  for (int rho = warp; rho < p.R; rho += kConsumers / 32) {
-    float M = -INFINITY;
-    for (int sp = lane; sp < nsplit; sp += 32) M = fmaxf(M, p.part_lse[prow(rho, sp)]);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float z = 0.f;
-    for (int sp = lane; sp < nsplit; sp += 32) {
-      const float l = p.part_lse[prow(rho, sp)];
-      z += (M == -INFINITY || l == -INFINITY) ? 0.f : expf(l - M);
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) z += __shfl_xor_sync(0xffffffffu, z, o);
-    if (lane == 0) {
-      rowm[rho] = M;
-      rowz[rho] = z;
-    }
-  }
-  consumer_sync();
-  for (int idx = tid; idx < p.R * (D / 4); idx += kConsumers) {
+  for (int idx = threadIdx.x; idx < p.R * (D / 4); idx += kConsumers) {
     const int rho = idx / (D / 4), d4 = idx % (D / 4);
-    const float M = rowm[rho], z = rowz[rho];
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (z > 0.f) {
-      for (int s0 = 0; s0 < nsplit; s0 += 8) {
-        float4 v[8];
-        float wv[8];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int sp = s0 + j;
-          const float l = (sp < nsplit) ? p.part_lse[prow(rho, sp)] : -INFINITY;
-          wv[j] = (l == -INFINITY) ? 0.f : expf(l - M);
-          v[j] = (sp < nsplit) ? reinterpret_cast<const float4*>(p.part_o + prow(rho, sp) * D)[d4]
-                               : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          acc.x += wv[j] * v[j].x;
-          acc.y += wv[j] * v[j].y;
-          acc.z += wv[j] * v[j].z;
-          acc.w += wv[j] * v[j].w;
-        }
-      }
-    }
-    const float inv = (z > 0.f) ? 1.f / z : 0.f;
     const int t = rho / p.g, h = kvh * p.g + rho % p.g;
+    const size_t row0 = (static_cast<size_t>(b) * p.Hq + h) * p.nsplit;
+    float lse;
+    const float4 o = lse_combine<8>(
+        p.nsplit, [&](int sp) { return p.part_lse[(row0 + sp) * p.T + t]; },
+        [&](int sp) { return reinterpret_cast<const float4*>(p.part_o + ((row0 + sp) * p.T + t) * D)[d4]; },
+        &lse);
     __nv_bfloat16* dst = p.o_merged + ((static_cast<size_t>(b) * p.T + t) * p.Hq + h) * D + 4 * d4;
     uint2 pk;
-    pk.x = pack_bf16x2(acc.x * inv, acc.y * inv);
-    pk.y = pack_bf16x2(acc.z * inv, acc.w * inv);
+    pk.x = pack_bf16x2(o.x, o.y);
+    pk.y = pack_bf16x2(o.z, o.w);
     *reinterpret_cast<uint2*>(dst) = pk;
-    if (d4 == 0 && p.lse_merged)
-      p.lse_merged[(static_cast<size_t>(b) * p.Hq + h) * p.T + t] = (z > 0.f) ? M + logf(z) : -INFINITY;
+    if (d4 == 0 && p.lse_merged) p.lse_merged[(static_cast<size_t>(b) * p.Hq + h) * p.T + t] = lse;
   }
 }
 
@@ -312,6 +267,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     issued = 0;
   }
   __syncthreads();
+  // the next kernel in the stream may be scheduled as this one's CTAs exit
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   if (warp == 4) {
     // ------------------------------------------------------------ producer
@@ -319,6 +276,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
       prefetch_tmap(&p.tmK);
       prefetch_tmap(&p.tmV);
     }
+    // every global access of this call follows the previous kernel's end
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int row0 = p.L + p.tail_len;  // cache row of new token 0
     int gt = 0;  // tiles issued over all units of this CTA
     bool stop = false;
@@ -387,6 +346,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     const int r0 = gq, r1 = gq + 8;
     const int g = p.g;
     const float c = p.scale_log2;
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      // the workspace header this call counts in, for star_device_status to
+      // clear after a device error
+      p.status[1] = p.header_bytes;
+    }
     uint32_t qf[kKSteps][4];
     int q_bh = -1;
     int gt = 0;  // tiles consumed over all units of this CTA
@@ -399,26 +364,42 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
       if (bh != q_bh) {
         // rows rho = t * g + hh of this GQA group (rows >= R are zero padding):
         // rotate them here (shared RoPE arithmetic, bit-identical to the
-        // RoPE kernel) into the free combine buffer, then take fragments
+        // RoPE kernel) into the free combine buffer, then take fragments.
+        // cos/sin (fp64) of each (token, frequency) pair are computed once,
+        // kTabPairs at a time, into the buffer after the rows: the g rows of
+        // a token share them.
         uint16_t* qs = reinterpret_cast<uint16_t*>(comb);  // [kDecRows][D] bf16 bits
-        for (int e = threadIdx.x; e < kDecRows * (D / 2); e += kConsumers) {
+        double* tcos = reinterpret_cast<double*>(qs + kDecRows * D);
+        double* tsin = tcos + kTabPairs;
+        constexpr int kTabTok = kTabPairs / (D / 2);       // tokens per table round
+        for (int e = p.R * (D / 2) + threadIdx.x; e < kDecRows * (D / 2); e += kConsumers) {
           const int rho = e / (D / 2), i = e % (D / 2);
-          uint32_t y0 = 0, y1 = 0;
-          if (rho < p.R) {
-            const int t = rho / g, hh = rho % g;
+          qs[rho * D + i] = 0;
+          qs[rho * D + i + D / 2] = 0;
+        }
+        for (int t0 = 0; t0 < p.T; t0 += kTabTok) {
+          const int tn = imin(kTabTok, p.T - t0);
+          for (int e = threadIdx.x; e < tn * (D / 2); e += kConsumers)
+            rope_angle(static_cast<long long>(p.q_pos0) + t0 + e / (D / 2),
+                       p.inv_freq[e % (D / 2)], &tcos[e], &tsin[e]);
+          // global memory only after the previous kernel's end (no-op after
+          // the first time)
+          asm volatile("griddepcontrol.wait;" ::: "memory");
+          consumer_sync();
+          for (int e = threadIdx.x; e < tn * g * (D / 2); e += kConsumers) {
+            const int rl = e / (D / 2), i = e % (D / 2);
+            const int tl = rl / g, rho = t0 * g + rl;
             const __nv_bfloat16* src =
-                p.q_new + ((static_cast<size_t>(b) * p.T + t) * p.Hq + kvh * g + hh) * D;
-            double c64, s64;
-            rope_angle(static_cast<long long>(p.q_pos0) + t, p.inv_freq[i], &c64, &s64);
+                p.q_new + ((static_cast<size_t>(b) * p.T + t0 + tl) * p.Hq + kvh * g + rl % g) * D;
+            const double c64 = tcos[tl * (D / 2) + i], s64 = tsin[tl * (D / 2) + i];
             const float a = __bfloat162float(src[i]), bb = __bfloat162float(src[i + D / 2]);
             const float c32 = static_cast<float>(c64), s32 = static_cast<float>(s64);
-            y0 = rope_rotate_bf16(a, bb, c32, s32, c64, s64, true);
-            y1 = rope_rotate_bf16(a, bb, c32, s32, c64, s64, false);
+            qs[rho * D + i] = static_cast<uint16_t>(rope_rotate_bf16(a, bb, c32, s32, c64, s64, true));
+            qs[rho * D + i + D / 2] =
+                static_cast<uint16_t>(rope_rotate_bf16(a, bb, c32, s32, c64, s64, false));
           }
-          qs[rho * D + i] = static_cast<uint16_t>(y0);
-          qs[rho * D + i + D / 2] = static_cast<uint16_t>(y1);
+          consumer_sync();  // the table is rewritten by the next round
         }
-        consumer_sync();
 #pragma unroll
         for (int kk = 0; kk < kKSteps; ++kk) {
           const int c0 = 16 * kk + 2 * t4;
@@ -598,21 +579,25 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
         int first, count;
         split_chunks(p, cr.split, &first, &count);
         __threadfence();
-        flag_last = (atomicAdd(&p.counters[bh * p.nsplit + cr.split], 1) == count - 1);
+        // wraps to 0 on the last arrival: the counter is zero again for the next call
+        flag_last = (atomicInc(reinterpret_cast<unsigned*>(&p.counters[bh * p.nsplit + cr.split]),
+                               static_cast<unsigned>(count - 1)) == static_cast<unsigned>(count - 1));
         __threadfence();
       }
       consumer_sync();
       if (flag_last) {
-        reduce_split<D>(p, bh, cr.split, comb);
+        reduce_split<D>(p, bh, cr.split);
         consumer_sync();
         if (p.o_merged != nullptr) {
           if (threadIdx.x == 0) {
             __threadfence();
-            flag_last = (atomicAdd(&p.head_counters[bh], 1) == p.n);
+            flag_last = (atomicInc(reinterpret_cast<unsigned*>(&p.head_counters[bh]),
+                                   static_cast<unsigned>(p.nsplit - 1)) ==
+                         static_cast<unsigned>(p.nsplit - 1));
             __threadfence();
           }
           consumer_sync();
-          if (flag_last) merge_head<D>(p, bh, comb);
+          if (flag_last) merge_head<D>(p, bh);
           consumer_sync();
         }
       }
@@ -644,11 +629,21 @@ cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t stream) {
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = imin(units, 2 * sms);  // persistent: two CTAs per SM
-  if (D == 128)
-    decode_kernel<128><<<grid, kDecThreads, smem, stream>>>(p);
-  else
-    decode_kernel<64><<<grid, kDecThreads, smem, stream>>>(p);
-  return cudaGetLastError();
+  // programmatic dependent launch: the kernel may start (barriers, tensor
+  // maps, the cos/sin table) while the previous kernel in the stream drains;
+  // it waits for that kernel's completion before touching global memory
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr_pdl[1];
+  attr_pdl[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr_pdl[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kDecThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cfg.attrs = attr_pdl;
+  cfg.numAttrs = 1;
+  return (D == 128) ? cudaLaunchKernelEx(&cfg, decode_kernel<128>, p)
+                    : cudaLaunchKernelEx(&cfg, decode_kernel<64>, p);
 }
 
 }  // namespace star

@@ -96,7 +96,8 @@ struct DecodeParams {
   float* lse_merged;        // nullable: [B, Hq, T]
   float* part_o;   // [B, Hq, nsplit, T, D]
   float* part_lse; // [B, Hq, nsplit, T]
-  int* status;
+  int* status;            // status word; status[1] receives header_bytes
+  int header_bytes;       // workspace bytes holding the status block and the counters
   float scale_log2, scale_ln;
 };
 size_t decode_smem_bytes(int D);

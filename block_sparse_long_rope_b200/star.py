@@ -296,6 +296,7 @@ def star_debug_index(L, block_len, anchor_len, device="cuda", stream=None):
 
 
 def alloc_workspace(nbytes, device="cuda"):
-    """A caller-owned workspace (the library itself allocates nothing)."""
+    """A caller-owned, zero-filled workspace (the library itself allocates
+    nothing; a workspace must be zero before its first use)."""
     n = max(256, (int(nbytes) + 255) // 256 * 256)
-    return torch.empty(n, dtype=torch.uint8, device=device)
+    return torch.zeros(n, dtype=torch.uint8, device=device)

@@ -36,6 +36,18 @@
  *   - Device errors found inside kernels (a bounded wait that gave up, an
  *     index outside its buffer) are recorded in a status word at the start of
  *     the call's workspace and read back by star_device_status.
+ *   - A workspace must be zero-filled once before its first use. After that
+ *     the library keeps it consistent: status bits are sticky (calls OR them
+ *     in, only star_device_status reads and clears them), and the counters of
+ *     the decode path, which every Phase-2 call keeps at the start of its
+ *     workspace, return to zero at the end of every call (after a device
+ *     error star_device_status clears them too). A workspace that decode
+ *     calls use may be shared with other Phase-2 calls of the same B, Hkv,
+ *     Lcap and block_len; before any other reuse it must be zero-filled
+ *     again. No call resets the workspace, so consecutive decode kernels run
+ *     back to back: the decode kernel is launched as a programmatic dependent
+ *     launch and waits for the previous kernel of the stream before its first
+ *     global memory access.
  */
 #ifndef STAR_H_
 #define STAR_H_

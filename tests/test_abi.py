@@ -53,9 +53,12 @@ def test_workspace_sizes(lib):
     # Phase 1: status header + rotated Q (bf16)
     assert lib.star_phase1_workspace_bytes(1, 2048, 4, 64) == 256 + 2048 * 4 * 64 * 2
     assert lib.star_phase1_workspace_bytes(2, 1000, 3, 128) >= 256 + 2 * 1000 * 3 * 128 * 2
-    # Phase 2 query chunk (tensor-core path): header + rotated q only
+    # Phase 2 query chunk (tensor-core path): the decode header (status block,
+    # split and head counters, kept on every Phase-2 path) + rotated q only
     chunk = lib.star_phase2_workspace_bytes(1, 128, 32, 8, 128, 16384 + 192, 4096)
-    assert chunk == 256 + 128 * 32 * 128 * 2
+    splits = -(-(16384 + 192) // 4096) + 1
+    header = 256 + (-(-(8 * splits * 4) // 256)) * 256 + 256
+    assert chunk == header + 128 * 32 * 128 * 2
     # decode path adds chunk scratch
     dec = lib.star_phase2_workspace_bytes(1, 1, 32, 8, 128, 16384 + 192, 4096)
     assert dec > 256 + 32 * 128 * 2

@@ -103,7 +103,11 @@ def run_flow(B, L, Hq, Hkv, D, b, a, theta, Ts, seed):
         assert ns2 == n + 1
         assert max_abs(to64(om2).transpose(0, 2, 1, 3).reshape(-1, D), mo) <= TOL_O
         assert max_abs(to64(lm2).reshape(-1), ml) <= TOL_LSE
-        assert torch.equal(po2, po) and torch.equal(pl2, pl)
+        # the split partials are the same quantities; on the decode path the
+        # fused call streams each split's chunks through an online softmax
+        # instead of a max-first reduction, so they agree to fp32 rounding
+        assert max_abs(to64(po2), to64(po)) <= 1e-4
+        assert max_abs(to64(pl2), to64(pl)) <= 1e-4
         # the appended cache rows hold the rotated new keys
         kref = orc.rope(kt.cpu(), np.arange(L + tail, L + tail + T), theta, round_out=True)
         kgot = to64(kc[:, :, L + tail:L + tail + T]).transpose(0, 2, 1, 3)
