@@ -223,6 +223,75 @@ __device__ void merge_head(const DecodeParams& p, int bh) {
   }
 }
 
+// Combine of the four consumer warps' partials of one unit (rows r0/r1 of
+// this lane, 16 keys per warp) into the chunk partial (ws_o, ws_lse). The
+// row statistics are exchanged first (cm, cl: [4][kDecRows]); each warp then
+// scales its own output by e^(m_w - M) / L (M the row max, L the combined
+// row sum), so the output columns are plain 4-term sums, kCols per round
+// through `co` ([4][kDecRows][kCols] floats), in a fixed order.
+template <int D, int kCols>
+__device__ __forceinline__ void combine_warps(const DecodeParams& p, float (&o)[D / 8][4],
+                                              float m0, float m1, float l0, float l1, float* cm,
+                                              float* cl, float* co, size_t base) {
+  const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+  const int t4 = lane & 3, r0 = lane >> 2, r1 = r0 + 8;
+  const float c = p.scale_log2;
+  if (t4 == 0) {
+    cm[warp * kDecRows + r0] = m0;
+    cm[warp * kDecRows + r1] = m1;
+    cl[warp * kDecRows + r0] = l0;
+    cl[warp * kDecRows + r1] = l1;
+  }
+  consumer_sync();
+  float sc[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int rho = k ? r1 : r0;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) M = fmaxf(M, cm[w * kDecRows + rho]);
+    float Ls = 0.f, mine = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const float e = ex2_approx((cm[w * kDecRows + rho] - M) * c);
+        Ls += e * cl[w * kDecRows + rho];
+        if (w == warp) mine = e;
+      }
+    }
+    sc[k] = (Ls > 0.f) ? mine / Ls : 0.f;
+    if (warp == 0 && t4 == 0 && rho < p.R)
+      p.ws_lse[base * kDecRows + rho] = (Ls > 0.f) ? M * p.scale_ln + logf(Ls) : -INFINITY;
+  }
+#pragma unroll
+  for (int dn = 0; dn < D / 8; ++dn) {
+    o[dn][0] *= sc[0];
+    o[dn][1] *= sc[0];
+    o[dn][2] *= sc[1];
+    o[dn][3] *= sc[1];
+  }
+#pragma unroll
+  for (int rd = 0; rd < D / kCols; ++rd) {
+#pragma unroll
+    for (int dn = rd * (kCols / 8); dn < (rd + 1) * (kCols / 8); ++dn) {
+      const int d = 8 * dn + 2 * t4 - rd * kCols;
+      co[(warp * kDecRows + r0) * kCols + d] = o[dn][0];
+      co[(warp * kDecRows + r0) * kCols + d + 1] = o[dn][1];
+      co[(warp * kDecRows + r1) * kCols + d] = o[dn][2];
+      co[(warp * kDecRows + r1) * kCols + d + 1] = o[dn][3];
+    }
+    consumer_sync();
+    for (int idx = threadIdx.x; idx < p.R * kCols; idx += kConsumers) {
+      const int rho = idx / kCols, dc = idx % kCols;
+      float out = 0.f;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) out += co[(w * kDecRows + rho) * kCols + dc];
+      p.ws_o[(base * kDecRows + rho) * D + rd * kCols + dc] = out;
+    }
+    consumer_sync();
+  }
+}
+
 // Persistent split-KV decode. CTA c owns the contiguous unit range
 // [c*U/G, (c+1)*U/G) of the U = B*Hkv*chunks_per_head (head, chunk) units.
 // The producer warp streams every tile of every unit through one ring; the
@@ -530,46 +599,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
       l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
 
       // ---- combine the four warps' partials, kCombCols columns per round
-      const size_t base = static_cast<size_t>(bh) * p.chunks_per_head + cidx;
-      if (t4 == 0) {
-        cm[warp * kDecRows + r0] = m0;
-        cm[warp * kDecRows + r1] = m1;
-        cl[warp * kDecRows + r0] = l0;
-        cl[warp * kDecRows + r1] = l1;
-      }
-#pragma unroll
-      for (int rd = 0; rd < D / kCombCols; ++rd) {
-#pragma unroll
-        for (int dn = rd * (kCombCols / 8); dn < (rd + 1) * (kCombCols / 8); ++dn) {
-          const int d = 8 * dn + 2 * t4 - rd * kCombCols;
-          co[(warp * kDecRows + r0) * kCombCols + d] = o[dn][0];
-          co[(warp * kDecRows + r0) * kCombCols + d + 1] = o[dn][1];
-          co[(warp * kDecRows + r1) * kCombCols + d] = o[dn][2];
-          co[(warp * kDecRows + r1) * kCombCols + d + 1] = o[dn][3];
-        }
-        consumer_sync();
-        for (int idx = threadIdx.x; idx < p.R * kCombCols; idx += kConsumers) {
-          const int rho = idx / kCombCols, dc = idx % kCombCols;
-          float M = -INFINITY;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) M = fmaxf(M, cm[w * kDecRows + rho]);
-          float out = 0.f, lse = -INFINITY;
-          if (M != -INFINITY) {
-            float Ls = 0.f, acc = 0.f;
-#pragma unroll
-            for (int w = 0; w < 4; ++w) {
-              const float e = ex2_approx((cm[w * kDecRows + rho] - M) * c);
-              Ls += e * cl[w * kDecRows + rho];
-              acc += e * co[(w * kDecRows + rho) * kCombCols + dc];
-            }
-            out = acc / Ls;
-            lse = M * p.scale_ln + logf(Ls);
-          }
-          p.ws_o[(base * kDecRows + rho) * D + rd * kCombCols + dc] = out;
-          if (rd == 0 && dc == 0) p.ws_lse[base * kDecRows + rho] = lse;
-        }
-        consumer_sync();
-      }
+      combine_warps<D, kCombCols>(p, o, m0, m1, l0, l1, cm, cl, co,
+                                  static_cast<size_t>(bh) * p.chunks_per_head + cidx);
       // ---- the CTA completing a split reduces it; the one completing a head
       // merges it. After the consumer barrier one thread publishes the CTA's
       // writes (fence, then count itself in) and, if last, fences again so
