@@ -276,42 +276,94 @@ def run_star(args, w, rank, world, local_rank):
         [elapsed_ms, p1_ms, chunk_ms, dec_ms], dev, world)
 
     # ---- end to end through the public API with host buffers ----------------
+    # Every step uploads its inputs from pinned host memory, runs the layer
+    # and reads its results back. Steps are pipelined over three streams (as a
+    # serving loop would run them): the upload of step i+1 overlaps the
+    # compute of step i and the read-back of step i-1. Two layers (caches,
+    # outputs) and two device input sets alternate, so no step waits on a
+    # buffer another step still uses except through the events below.
     host_ctx = [t.cpu().pin_memory() for t in ctx]
     host_calls = [tuple(x.cpu().pin_memory() for x in c[:3]) + (c[3],) for c in calls]
-    dev_ctx = [torch.empty_like(t) for t in ctx]
-    dev_calls = [tuple(torch.empty_like(x) for x in c[:3]) + (c[3],) for c in calls]
-    host_o = torch.empty(layer.buf.o.shape, dtype=torch.bfloat16).pin_memory()
+    layers2 = [layer, StarLayer(w, device=dev)]
+    dev_sets = [([torch.empty_like(t) for t in ctx],
+                 [tuple(torch.empty_like(x) for x in c[:3]) + (c[3],) for c in calls])
+                for _ in range(2)]
+    # the step's result read back is the last generated token's attention
+    # output; the Phase-1 output stays on the device (a decoder's next layer
+    # consumes it there)
     host_dec = torch.empty((w.B, 1, w.Hq, w.D), dtype=torch.bfloat16).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_ctx) + \
         sum(x.numel() * x.element_size() for c in host_calls for x in c[:3])
-    d2h = host_o.numel() * 2 + host_dec.numel() * 2
+    d2h = host_dec.numel() * 2
+    s_up, s_comp, s_down = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev_up = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_down = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        for d, h in zip(dev_ctx, host_ctx):
-            d.copy_(h, non_blocking=True)
-        for dc, hc in zip(dev_calls, host_calls):
-            for d, h in zip(dc[:3], hc[:3]):
-                d.copy_(h, non_blocking=True)
-        layer.encode(*dev_ctx)
+    def compute(k):
+        lay, (dctx, dcalls) = layers2[k], dev_sets[k]
+        lay.encode(*dctx)
         out = None
-        for (q2, k2, v2, tail) in dev_calls:
-            out = layer.attend(q2, k2, v2, tail)
-        host_o.copy_(layer.buf.o, non_blocking=True)
-        host_dec.copy_(out[0], non_blocking=True)
+        for (q2, k2, v2, tail) in dcalls:
+            out = lay.attend(q2, k2, v2, tail)
+        return out
 
-    for _ in range(max(1, args.warmup // 2)):
-        e2e_step()
+    replay = [None, None]  # with --graph: the compute of each buffer set as a CUDA graph
+
+    def e2e_step(i):
+        k = i % 2
+        lay, (dctx, dcalls) = layers2[k], dev_sets[k]
+        s_up.wait_event(ev_comp[k])        # step i-2 no longer reads these inputs
+        with torch.cuda.stream(s_up):
+            for d, h in zip(dctx, host_ctx):
+                d.copy_(h, non_blocking=True)
+            for dc, hc in zip(dcalls, host_calls):
+                for d, h in zip(dc[:3], hc[:3]):
+                    d.copy_(h, non_blocking=True)
+            ev_up[k].record(s_up)
+        s_comp.wait_event(ev_up[k])
+        s_comp.wait_event(ev_down[k])      # step i-2's outputs have been read back
+        with torch.cuda.stream(s_comp):
+            if replay[k] is not None:
+                replay[k][0].replay()
+                out = replay[k][1]
+            else:
+                out = compute(k)
+            ev_comp[k].record(s_comp)
+        s_down.wait_event(ev_comp[k])
+        with torch.cuda.stream(s_down):
+            host_dec.copy_(out[0], non_blocking=True)
+            ev_down[k].record(s_down)
+
+    for i in range(max(2, args.warmup // 2)):
+        e2e_step(i)
     torch.cuda.synchronize()
+    if args.graph:
+        for k in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=s_comp):
+                out_k = compute(k)
+            replay[k] = (g, out_k)
+        for i in range(2):
+            e2e_step(i)
+        torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     s2 = torch.cuda.Event(enable_timing=True)
     e2 = torch.cuda.Event(enable_timing=True)
-    s2.record(stream)
-    for _ in range(args.steps):
-        e2e_step()
-    e2.record(stream)
+    s2.record(s_up)
+    s_comp.wait_event(s2)
+    s_down.wait_event(s2)
+    for i in range(args.steps):
+        e2e_step(i)
+    s_down.wait_event(ev_comp[(args.steps - 1) % 2])
+    e2.record(s_down)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks([s2.elapsed_time(e2)], dev, world)[0]
+    for lay in layers2:
+        star.star_device_status(lay.buf.ws1)
+        star.star_device_status(lay.buf.ws2)
+    del layers2[1], dev_sets, replay
 
     # ---- generalised prefix: Pulsar's layout on the same workload (a side
     # measurement outside the step: sink + 12.5% chunk summaries per block)
@@ -462,7 +514,14 @@ def run_star(args, w, rank, world, local_rank):
                      "traffic": phase1_traffic(w.name),
                      "traffic_unit": "bytes per launch (DRAM read + write, ncu)"},
         "e2e": {"value": round(job_value(w.B * w.L, world, e2e_ms / K), 1), "unit": "tok/s",
-                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)},
+                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+                "ms_per_step": round(e2e_ms / K, 4),
+                "note": "public API (StarLayer.encode/attend; with the default graph launch "
+                        "each buffer set's calls are captured once and replayed); every step "
+                        "uploads all its inputs (context Q/K/V and the new tokens) from pinned "
+                        "host memory and reads back its result, the last generated token's "
+                        "attention output (the Phase-1 output stays on the device for the next "
+                        "layer); steps pipelined over upload / compute / read-back streams"},
         "gpu_launches": launches * K,
         "clocks": clocks,
     }
@@ -541,11 +600,10 @@ def run_sharded(args, w, rank, world, local_rank):
     host_calls = [tuple(x.cpu().pin_memory() for x in c[:3]) + (c[3],) for c in calls]
     dev_ctx = [torch.empty_like(t) for t in ctx + anchor]
     dev_calls = [tuple(torch.empty_like(x) for x in c[:3]) + (c[3],) for c in calls]
-    host_o = torch.empty(layer.o.shape, dtype=torch.bfloat16).pin_memory()
     host_dec = torch.empty((w.B, 1, w.Hq, w.D), dtype=torch.bfloat16).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_ctx) + \
         sum(x.numel() * x.element_size() for c in host_calls for x in c[:3])
-    d2h = host_o.numel() * 2 + host_dec.numel() * 2
+    d2h = host_dec.numel() * 2  # the last generated token's attention output
 
     def e2e_step():
         for d, h in zip(dev_ctx, host_ctx):
@@ -557,7 +615,6 @@ def run_sharded(args, w, rank, world, local_rank):
         out = None
         for (q2, k2, v2, tail) in dev_calls:
             out = layer.attend(q2, k2, v2, tail)
-        host_o.copy_(layer.o, non_blocking=True)
         host_dec.copy_(out[0], non_blocking=True)
 
     for _ in range(max(1, args.warmup // 2)):
