@@ -345,8 +345,12 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
       prefetch_tmap(&p.tmK);
       prefetch_tmap(&p.tmV);
     }
-    // every global access of this call follows the previous kernel's end
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // Only a decode kernel starts this one before it ends (no other kernel of
+    // the library triggers its dependents), and a decode kernel never writes
+    // cache rows [0, L) or q: tiles of those rows are loaded at once; the
+    // tail rows (appended by the previous step) and the append wait for the
+    // previous kernel's end.
+    bool waited = false;
     const int row0 = p.L + p.tail_len;  // cache row of new token 0
     int gt = 0;  // tiles issued over all units of this CTA
     bool stop = false;
@@ -359,6 +363,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
       // tile (no other unit reads the row). The warp writes, every lane
       // fences its generic writes against the TMA (async proxy) reads.
       const int w_lo = imax(cr.k_lo, row0), w_hi = p.with_tail ? imin(cr.k_hi, row0 + p.T) : 0;
+      if (w_lo < w_hi && !waited) {
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        waited = true;
+      }
       if (w_lo < w_hi) {
         const int b = bh / p.Hkv, kvh = bh % p.Hkv;
         for (int r = w_lo; r < w_hi; ++r) {
@@ -381,6 +389,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
         __syncwarp();
       }
       for (int it = 0; it < nt; ++it, ++gt) {
+        if (!waited && cr.k_lo + (it + 1) * kDecTile > p.L) {  // reaches the tail rows
+          asm volatile("griddepcontrol.wait;" ::: "memory");
+          waited = true;
+        }
         int ok = 1;
         if (lane == 0) {
           const int st = gt % kDecStages, use = gt / kDecStages;
@@ -415,12 +427,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     const int r0 = gq, r1 = gq + 8;
     const int g = p.g;
     const float c = p.scale_log2;
-    if (blockIdx.x == 0 && threadIdx.x == 0) {
-      asm volatile("griddepcontrol.wait;" ::: "memory");
-      // the workspace header this call counts in, for star_device_status to
-      // clear after a device error
-      p.status[1] = p.header_bytes;
-    }
     uint32_t qf[kKSteps][4];
     int q_bh = -1;
     int gt = 0;  // tiles consumed over all units of this CTA
@@ -451,9 +457,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
           for (int e = threadIdx.x; e < tn * (D / 2); e += kConsumers)
             rope_angle(static_cast<long long>(p.q_pos0) + t0 + e / (D / 2),
                        p.inv_freq[e % (D / 2)], &tcos[e], &tsin[e]);
-          // global memory only after the previous kernel's end (no-op after
-          // the first time)
-          asm volatile("griddepcontrol.wait;" ::: "memory");
           consumer_sync();
           for (int e = threadIdx.x; e < tn * g * (D / 2); e += kConsumers) {
             const int rl = e / (D / 2), i = e % (D / 2);
@@ -593,6 +596,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
       // all four consumer warps decide together whether to stop (a warp still
       // inside the tile loop would otherwise miss the named barriers below)
       if (consumer_sync_or(abort_flag)) break;
+      // the first global write of this call (the previous kernel may still be
+      // reducing its own partials from the workspace) follows its end
+      asm volatile("griddepcontrol.wait;" ::: "memory");
+      if (blockIdx.x == 0 && threadIdx.x == 0 && u == u_begin)
+        p.status[1] = p.header_bytes;  // the header this call counts in, for star_device_status
       l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
       l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
       l1 += __shfl_xor_sync(0xffffffffu, l1, 1);

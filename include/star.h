@@ -46,8 +46,12 @@
  *     Lcap and block_len; before any other reuse it must be zero-filled
  *     again. No call resets the workspace, so consecutive decode kernels run
  *     back to back: the decode kernel is launched as a programmatic dependent
- *     launch and waits for the previous kernel of the stream before its first
- *     global memory access.
+ *     launch. Only a decode kernel can start it early, so it streams cache
+ *     rows [0, L) and reads q before that kernel has finished, and waits for
+ *     it before touching the tail rows and before its first write.
+ *     Consecutive decode calls on one cache must therefore keep the context
+ *     length L and grow only the tail. This is how Phase 2 proceeds: the
+ *     context is fixed after Phase 1.
  */
 #ifndef STAR_H_
 #define STAR_H_
