@@ -194,13 +194,14 @@ int decode_chunk(int B, int Hkv, int L, int b, int n, int nsplit, int tail_plus_
   return static_cast<int>(chunk_tiles) * tile;
 }
 
-// Bytes of the zeroed header of a decode workspace: the status word, one
-// finished-chunk counter per (batch, KV head, split), then one finished-split
-// counter per (batch, KV head).
+// Bytes of the finished-chunk counters: one per (batch, KV head, split).
 size_t decode_split_counter_bytes(int B, int Hkv, int Lcap, int block_len) {
   const long long nsplit_cap = ceil_div(Lcap, block_len) + 1;
   return align_up((size_t)B * Hkv * nsplit_cap * sizeof(int));
 }
+// Bytes of the header of a Phase-2 workspace (zero between calls): the
+// status block, the finished-chunk counters, then one finished-split counter
+// per (batch, KV head).
 size_t decode_header_bytes(int B, int Hkv, int Lcap, int block_len) {
   return star::kStatusBytes + decode_split_counter_bytes(B, Hkv, Lcap, block_len) +
          align_up((size_t)B * Hkv * sizeof(int));

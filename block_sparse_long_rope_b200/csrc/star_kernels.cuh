@@ -90,8 +90,8 @@ struct DecodeParams {
   int nc_full, nc_last, nc_tail, chunks_per_head;  // chunk counts per split kind
   float* ws_o;     // [B*Hkv, chunks_per_head, kDecRows, D] chunk-normalised output
   float* ws_lse;   // [B*Hkv, chunks_per_head, kDecRows]
-  int* counters;   // [B*Hkv, nsplit] finished chunks per split, zero at launch
-  int* head_counters;  // [B*Hkv] finished splits per (batch, KV head), zero at launch
+  int* counters;   // [B*Hkv, nsplit] finished chunks per split; zero between calls
+  int* head_counters;  // [B*Hkv] finished splits per (batch, KV head); zero between calls
   __nv_bfloat16* o_merged;  // nullable: [B, T, Hq, D] merged output (also needs head_counters)
   float* lse_merged;        // nullable: [B, Hq, T]
   float* part_o;   // [B, Hq, nsplit, T, D]

@@ -177,7 +177,9 @@ star_status star_phase1_encode_ext(const void* q, const void* k, const void* v, 
 
 /* Workspace bytes star_phase2_partial needs for up to T new tokens with a
  * cache of capacity Lcap (context L plus tail) split into blocks of
- * block_len. */
+ * block_len: the header (256-byte status block, then the decode path's
+ * split and head counters, kept on every Phase-2 path), the rotated q and,
+ * on the decode path (T * Hq / Hkv <= 16), the chunk partials. */
 size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lcap, int block_len);
 
 /*
@@ -334,11 +336,13 @@ star_status star_linear(const void* x, const void* w, void* y, int M, int N, int
                         void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /*
- * star_device_status — synchronises `cuda_stream`, then reads and clears the
- * status word at the start of `workspace` (a workspace passed to
- * star_phase1_encode or star_phase2_partial). Returns STAR_OK,
- * STAR_ERR_DEVICE_TIMEOUT or STAR_ERR_DEVICE_BOUNDS (message in
- * star_last_error), or STAR_ERR_CUDA.
+ * star_device_status — synchronises `cuda_stream`, then reads the status
+ * bits at the start of `workspace` (a workspace passed to any call; the bits
+ * are sticky since the last read) and clears them. After a device error it
+ * also clears the decode counters (the header size the last decode call
+ * recorded in the status block), since an aborted call may leave them
+ * non-zero. Returns STAR_OK, STAR_ERR_DEVICE_TIMEOUT or STAR_ERR_DEVICE_BOUNDS
+ * (message in star_last_error), or STAR_ERR_CUDA.
  */
 star_status star_device_status(void* workspace, void* cuda_stream);
 
