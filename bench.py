@@ -141,21 +141,31 @@ def oracle_sample(w, budget_s=15.0, seed=0):
     return est_step, sample, t_p1 + t_dec
 
 
+def code_digest(paths):
+    """sha256 of the given sources with comments and whitespace removed, so
+    that only a change of the code itself marks a capture as stale."""
+    import hashlib
+    import re
+
+    h = hashlib.sha256()
+    for src in paths:
+        with open(os.path.join(ROOT, src)) as g:
+            text = g.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(re.sub(r"\s+", "", text).encode())
+    return h.hexdigest()
+
+
 def phase1_traffic(workload):
     """DRAM bytes (read + write) of one star_phase1_encode launch from the ncu
-    capture recorded under profiles/, if the kernel sources are still the ones
-    that were profiled; None otherwise (the counters no longer apply)."""
-    import hashlib
-
+    capture recorded under profiles/, if the kernel code is still the code
+    that was profiled; None otherwise (the counters no longer apply)."""
     path = os.path.join(ROOT, "profiles", f"phase1_traffic_{workload}.json")
     try:
         with open(path) as f:
             rec = json.load(f)
-        h = hashlib.sha256()
-        for src in rec["sources"]:
-            with open(os.path.join(ROOT, src), "rb") as g:
-                h.update(g.read())
-        if h.hexdigest() != rec["sources_sha256"]:
+        if code_digest(rec["sources"]) != rec["code_sha256"]:
             return None
         return int(rec["traffic_bytes_per_launch"])
     except (OSError, KeyError, ValueError):
