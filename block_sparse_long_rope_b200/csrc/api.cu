@@ -133,6 +133,8 @@ star_status map_cache(CUtensorMap* m, const void* base, int BH, int Lcap, int va
 // ---- shared argument checks ----------------------------------------------------
 star_status check_heads(int B, int Hq, int Hkv, int D) {
   if (B < 1 || Hq < 1 || Hkv < 1) return fail(STAR_ERR_INVALID_ARG, "B, Hq, Hkv must be >= 1");
+  if (Hq > star::kMaxHeads)
+    return fail(STAR_ERR_INVALID_ARG, "Hq (%d) must be <= %d", Hq, star::kMaxHeads);
   if (Hq % Hkv != 0) return fail(STAR_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
   if (D != 64 && D != 128) return fail(STAR_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", D);
   return STAR_OK;
@@ -239,7 +241,8 @@ star_status star_rope(const void* x, const int64_t x_stride[3], void* y, const i
                       const int32_t* pos, int64_t pos0, int B, int S, int H, int D, double theta,
                       void* cuda_stream) {
   if (!x_stride || !y_stride) return fail(STAR_ERR_INVALID_ARG, "stride arrays are NULL");
-  if (B < 0 || S < 0 || H < 1) return fail(STAR_ERR_INVALID_ARG, "bad shape B=%d S=%d H=%d", B, S, H);
+  if (B < 0 || S < 0 || H < 1 || H > star::kMaxHeads)
+    return fail(STAR_ERR_INVALID_ARG, "bad shape B=%d S=%d H=%d (H <= %d)", B, S, H, star::kMaxHeads);
   if (D != 64 && D != 128) return fail(STAR_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", D);
   if (!(theta > 0.0)) return fail(STAR_ERR_INVALID_ARG, "theta must be > 0");
   star_status s;

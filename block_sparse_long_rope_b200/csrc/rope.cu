@@ -38,9 +38,10 @@ constexpr int kRopeThreads = 256;
 constexpr int kTokPerCta = 8;
 }  // namespace
 
+template <int D>
 __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constant__ RopeParams p) {
+  constexpr int kHalf = D / 2, kCpr = kHalf / 8;  // 16-byte chunks per half row
   const RopeJob& job = p.job[blockIdx.z];
-  const int D = p.D, half = D / 2, cpr = half / 8;  // 16-byte chunks per half row
   const int tok0 = blockIdx.x * kTokPerCta;
   const int b = blockIdx.y;
   const int ntok = imin(kTokPerCta, p.S - tok0);
@@ -63,10 +64,10 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
     __syncthreads();
   }
   if (job.rotate) {
-    for (int e = threadIdx.x; e < ntok * half; e += blockDim.x) {
-      int t = e / half, i = e % half;
-      int s = tok0 + t;
-      long long pos = p.pos ? static_cast<long long>(p.pos[s]) : p.pos0 + s;
+    for (int e = threadIdx.x; e < ntok * kHalf; e += kRopeThreads) {
+      const int t = e / kHalf, i = e % kHalf;
+      const int s = tok0 + t;
+      const long long pos = p.pos ? static_cast<long long>(p.pos[s]) : p.pos0 + s;
       double sn, cs;
       rope_angle(pos, p.inv_freq[i], &cs, &sn);
       s_cos[t][i] = cs;
@@ -77,12 +78,16 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
     __syncthreads();
   }
 
-  const int units = ntok * job.H * cpr;  // (token, head, chunk) triples
-  for (int u = threadIdx.x; u < units; u += blockDim.x) {
-    int c = u % cpr;
-    int h = (u / cpr) % job.H;
-    int t = u / (cpr * job.H);
-    int s = tok0 + t;
+  // units (token, head, chunk): the token by one multiply-high with a magic
+  // number (exact: u * per_tok < 2^32), head and chunk by constant shifts
+  const unsigned per_tok = static_cast<unsigned>(job.H) * kCpr;
+  const unsigned units = static_cast<unsigned>(ntok) * per_tok;
+  const unsigned magic = 0xFFFFFFFFu / per_tok + 1u;
+  for (unsigned u = threadIdx.x; u < units; u += kRopeThreads) {
+    const int t = static_cast<int>(__umulhi(u, magic));
+    const unsigned rem = u - static_cast<unsigned>(t) * per_tok;
+    const int h = static_cast<int>(rem / kCpr), c = static_cast<int>(rem % kCpr);
+    const int s = tok0 + t;
     __nv_bfloat16* yr = job.y + b * job.ys[0] + s * job.ys[1] + h * job.ys[2];
     const __nv_bfloat16* xr;
     if (!p.src) {
@@ -90,7 +95,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
     } else if (!s_ok[t]) {
       const uint4 z = make_uint4(0u, 0u, 0u, 0u);
       *reinterpret_cast<uint4*>(yr + 8 * c) = z;
-      *reinterpret_cast<uint4*>(yr + half + 8 * c) = z;
+      *reinterpret_cast<uint4*>(yr + kHalf + 8 * c) = z;
       continue;
     } else {
       const int r = s_row[t];
@@ -98,7 +103,7 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
                     : job.x2 + b * job.x2s[0] + (-1 - r) * job.x2s[1] + h * job.x2s[2];
     }
     uint4 lo = *reinterpret_cast<const uint4*>(xr + 8 * c);
-    uint4 hi = *reinterpret_cast<const uint4*>(xr + half + 8 * c);
+    uint4 hi = *reinterpret_cast<const uint4*>(xr + kHalf + 8 * c);
     if (job.rotate) {
       const uint32_t* pl = reinterpret_cast<const uint32_t*>(&lo);
       const uint32_t* ph = reinterpret_cast<const uint32_t*>(&hi);
@@ -106,22 +111,19 @@ __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constan
 #pragma unroll
       for (int w = 0; w < 4; ++w) {
         const int i0 = 8 * c + 2 * w;
-        const float a0 = bf16_lo(pl[w]), a1 = bf16_hi(pl[w]);
-        const float b0 = bf16_lo(ph[w]), b1 = bf16_hi(ph[w]);
-        ol[w] = rope_rotate_bf16(a0, b0, f_cos[t][i0], f_sin[t][i0], s_cos[t][i0], s_sin[t][i0], true) |
-                (rope_rotate_bf16(a1, b1, f_cos[t][i0 + 1], f_sin[t][i0 + 1], s_cos[t][i0 + 1],
-                                  s_sin[t][i0 + 1], true)
-                 << 16);
-        oh[w] = rope_rotate_bf16(a0, b0, f_cos[t][i0], f_sin[t][i0], s_cos[t][i0], s_sin[t][i0], false) |
-                (rope_rotate_bf16(a1, b1, f_cos[t][i0 + 1], f_sin[t][i0 + 1], s_cos[t][i0 + 1],
-                                  s_sin[t][i0 + 1], false)
-                 << 16);
+        const uint32_t p0 = rope_rotate_pair_bf16(bf16_lo(pl[w]), bf16_lo(ph[w]), f_cos[t][i0],
+                                                  f_sin[t][i0], &s_cos[t][i0], &s_sin[t][i0]);
+        const uint32_t p1 = rope_rotate_pair_bf16(bf16_hi(pl[w]), bf16_hi(ph[w]), f_cos[t][i0 + 1],
+                                                  f_sin[t][i0 + 1], &s_cos[t][i0 + 1],
+                                                  &s_sin[t][i0 + 1]);
+        ol[w] = __byte_perm(p0, p1, 0x5410);  // first outputs of both pairs
+        oh[w] = __byte_perm(p0, p1, 0x7632);  // second outputs
       }
       lo = make_uint4(ol[0], ol[1], ol[2], ol[3]);
       hi = make_uint4(oh[0], oh[1], oh[2], oh[3]);
     }
     *reinterpret_cast<uint4*>(yr + 8 * c) = lo;
-    *reinterpret_cast<uint4*>(yr + half + 8 * c) = hi;
+    *reinterpret_cast<uint4*>(yr + kHalf + 8 * c) = hi;
   }
 }
 
@@ -133,7 +135,10 @@ void rope_fill_freq(double* out, int D, double theta) {
 cudaError_t launch_rope(const RopeParams& p, int njobs, cudaStream_t stream) {
   if (njobs <= 0 || p.S <= 0 || p.B <= 0) return cudaSuccess;
   dim3 grid(ceil_div(p.S, kTokPerCta), p.B, njobs);
-  rope_kernel<<<grid, kRopeThreads, 0, stream>>>(p);
+  if (p.D == 128)
+    rope_kernel<128><<<grid, kRopeThreads, 0, stream>>>(p);
+  else
+    rope_kernel<64><<<grid, kRopeThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
 

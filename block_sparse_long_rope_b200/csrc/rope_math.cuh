@@ -54,4 +54,25 @@ __device__ __forceinline__ uint32_t rope_rotate_bf16(float a, float b, float c32
   return pack_bf16x2(f32_round_odd(yd), 0.f) & 0xFFFFu;
 }
 
+// Both outputs of one pair: low 16 bits the bf16 of a*c - b*s, high 16 bits
+// that of b*c + a*s, each correctly rounded exactly as rope_rotate_bf16 does.
+// The error bound is shared, and the fp64 cos/sin (c64, s64: read through
+// the pointers) are loaded only when a result is within the bound of a
+// rounding boundary.
+__device__ __forceinline__ uint32_t rope_rotate_pair_bf16(float a, float b, float c32, float s32,
+                                                          const double* c64, const double* s64) {
+  const float e = 2.3841858e-07f * (fabsf(a) + fabsf(b));
+  const float y0 = fmaf(a, c32, -(b * s32));
+  const float y1 = fmaf(b, c32, a * s32);
+  const uint32_t r0 = pack_bf16x2(y0 - e, y0 + e), r1 = pack_bf16x2(y1 - e, y1 + e);
+  uint32_t o0 = r0 & 0xFFFFu, o1 = r1 & 0xFFFFu;
+  const bool ok0 = o0 == (r0 >> 16), ok1 = o1 == (r1 >> 16);
+  if (!(ok0 && ok1)) {
+    const double ad = a, bd = b, cd = *c64, sd = *s64;
+    if (!ok0) o0 = pack_bf16x2(f32_round_odd(ad * cd - bd * sd), 0.f) & 0xFFFFu;
+    if (!ok1) o1 = pack_bf16x2(f32_round_odd(bd * cd + ad * sd), 0.f) & 0xFFFFu;
+  }
+  return o0 | (o1 << 16);
+}
+
 }  // namespace star

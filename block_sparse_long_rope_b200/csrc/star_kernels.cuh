@@ -12,6 +12,7 @@
 namespace star {
 
 // ---- RoPE / cache write ----------------------------------------------------
+constexpr int kMaxHeads = 2048;  // heads per call (keeps the RoPE kernel's unit index math in 32 bits)
 struct RopeJob {
   const __nv_bfloat16* x;
   __nv_bfloat16* y;

@@ -32,7 +32,8 @@
  *   - RoPE is rotate-half with base theta: pair (x_i, x_{i+D/2}) turns by the
  *     angle p * theta^(-2i/D); token t of the context sits at position t, so
  *     the anchor keeps positions 0..a-1 in every block.
- *   - Supported head_dim D: 64 and 128. Pointers must be 16-byte aligned.
+ *   - Supported head_dim D: 64 and 128; at most 2048 heads. Pointers must be
+ *     16-byte aligned.
  *   - Device errors found inside kernels (a bounded wait that gave up, an
  *     index outside its buffer) are recorded in a status word at the start of
  *     the call's workspace and read back by star_device_status.
