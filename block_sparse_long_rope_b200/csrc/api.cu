@@ -209,6 +209,38 @@ size_t decode_header_bytes(int B, int Hkv, int Lcap, int block_len) {
          align_up((size_t)B * Hkv * sizeof(int));
 }
 
+// Query chunks (tensor-core path): sub-splits per context block. A call with
+// fewer (split, query tile, head group) items than one wave of a B200 (148
+// CTAs) cuts every block into nsub equal sub-splits (a multiple of 128 keys,
+// at most 4), so more SMs share the work; the sub-split partials are then
+// reduced into the per-split partials. Only whole blocks (L a multiple of
+// block_len) and calls with the tail split are cut. Depends on the shape
+// only, so the workspace size can be computed without a device.
+int chunk_subsplits(int B, int Hq, int Hkv, int T, int L, int block_len, int with_tail) {
+  constexpr long long kWave = 148;
+  if (!with_tail || L % block_len != 0) return 1;
+  const int n = L / block_len;
+  const int g = Hq / Hkv, hpc = (g % 2 == 0) ? 2 : 1;
+  const long long per_split = (long long)B * Hkv * (g / hpc) * ceil_div(T, 128);
+  if ((n + 1) * per_split >= kWave) return 1;
+  int nsub = (int)std::min<long long>(4, (kWave - per_split) / (n * per_split));
+  while (nsub > 1 && block_len % (nsub * 128) != 0) --nsub;
+  return std::max(1, nsub);
+}
+
+// Workspace bytes of the sub-split partials of a query chunk, for the
+// largest count any context of at most Lcap rows can need.
+size_t chunk_scratch_bytes(int B, int T, int Hq, int Hkv, int D, int Lcap, int block_len) {
+  size_t best = 0;
+  for (int n = 1; (long long)n * block_len <= Lcap; ++n) {
+    const int nsub = chunk_subsplits(B, Hq, Hkv, T, n * block_len, block_len, 1);
+    if (nsub <= 1) continue;
+    const size_t rows = (size_t)B * Hq * (n * nsub + 1) * T;
+    best = std::max(best, align_up(rows * D * sizeof(float)) + align_up(rows * sizeof(float)));
+  }
+  return best;
+}
+
 bool use_decode_path(int T, int Hq, int Hkv) {
   const int g = Hq / Hkv;
   return T * g <= star::kDecRows;
@@ -461,7 +493,7 @@ size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lca
   // in front, so query-chunk and decode calls can share one workspace
   const size_t head = decode_header_bytes(B, Hkv, Lcap, block_len) + align_up((size_t)B * T * Hq * D * 2);
   if (use_decode_path(T, Hq, Hkv)) return head + decode_scratch_bytes(B, Hkv, D, Lcap, block_len);
-  return head;
+  return head + chunk_scratch_bytes(B, T, Hq, Hkv, D, Lcap, block_len);
 }
 
 }  // extern "C"
@@ -624,17 +656,32 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   ap.geom.T = T;
   ap.geom.tail_len = tail_len;
   ap.geom.tail = with_tail;
+  // sub-splits: their partials go to the workspace, then are reduced per split
+  const int nsub = chunk_subsplits(B, Hq, Hkv, T, L, block_len, with_tail);
+  ap.geom.nsub = nsub;
+  ap.geom.sub_len = block_len / nsub;
+  float* sub_o = part_o;
+  float* sub_lse = part_lse;
+  if (nsub > 1) {
+    const size_t rows = (size_t)B * Hq * (n * nsub + 1) * T;
+    sub_o = reinterpret_cast<float*>(ws + header + qrot_bytes);
+    sub_lse = reinterpret_cast<float*>(ws + header + qrot_bytes + align_up(rows * D * sizeof(float)));
+  }
   ap.mode = 1;
   ap.num_items = ap.geom.phase2_items();
   ap.qrows = T;
-  ap.nsplit = nsplit;
-  ap.part_o = part_o;
-  ap.part_lse = part_lse;
+  ap.nsplit = ap.geom.phase2_splits();
+  ap.part_o = sub_o;
+  ap.part_lse = sub_lse;
   ap.status = reinterpret_cast<int*>(ws);
   ap.scale_ln = (float)(1.0 / sqrt((double)D));
   ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   e = star::launch_attn(ap, D, st);
   if (e != cudaSuccess) return cuda_fail(e, "phase-2 chunk attention launch");
+  if (nsub > 1) {
+    e = star::launch_subsplit_reduce(sub_o, sub_lse, nsub, n, part_o, part_lse, B, T, Hq, D, st);
+    if (e != cudaSuccess) return cuda_fail(e, "sub-split reduce launch");
+  }
   if (o_merged) {
     star::MergeSegs segs{};
     segs.nseg = 1;

@@ -73,6 +73,7 @@ struct AttnGeom {
   // Phase 2 only
   int T, tail_len;
   int tail;             // 1: the call's cache holds the tail split (new tokens)
+  int nsub, sub_len;    // query chunks: sub-splits per context block, keys each
 
   __host__ __device__ int groups() const { return B * Hkv * ((Hq / Hkv) / hpc); }
   __host__ __device__ int qtiles_full() const { return ceil_div(imin(b, L), kTileM); }
@@ -134,10 +135,12 @@ struct AttnGeom {
   }
 
   // ---- Phase 2 (query chunk, partial mode) ---------------------------------
-  // Items: split-major (context blocks 0..n-1, then the tail), then query
-  // tile, then head group.
+  // Items: split-major (context blocks 0..n-1, each cut into nsub equal
+  // sub-splits of sub_len keys, then the tail), then query tile, then head
+  // group. Item split index s < n*nsub is sub-split s % nsub of block s / nsub.
   __host__ __device__ int phase2_qtiles() const { return ceil_div(T, kTileM); }
-  __host__ __device__ int phase2_items() const { return (n + tail) * phase2_qtiles() * groups(); }
+  __host__ __device__ int phase2_splits() const { return n * nsub + tail; }
+  __host__ __device__ int phase2_items() const { return phase2_splits() * phase2_qtiles() * groups(); }
   __host__ __device__ WorkItem phase2_item(int item) const {
     int G = groups(), nq = phase2_qtiles();
     int split = item / (nq * G);
@@ -151,8 +154,9 @@ struct AttnGeom {
     w.split = split;
     w.nspan = 1;
     w.span[1] = KvSpan{0, 0, 0, 0, 0, 0};
-    if (split < n) {
-      int s = split * b, e = imin(s + b, L);
+    if (split < n * nsub) {
+      const int blk = split / nsub, sub = split % nsub;
+      int s = blk * b + sub * sub_len, e = imin(imin(s + sub_len, (blk + 1) * b), L);
       w.span[0] = KvSpan{s, ceil_div(e - s, kTileN), s, e, 0, 0};
     } else {
       // tail keys [L, L + tail_len + T); this tile's last row sits at

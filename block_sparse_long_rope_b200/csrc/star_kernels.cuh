@@ -116,6 +116,9 @@ struct MergeSegs {
 cudaError_t launch_lse_merge(const float* part_o, const float* part_lse, const MergeSegs& segs,
                              __nv_bfloat16* o, float* lse, int B, int T, int Hq, int D,
                              cudaStream_t stream);
+cudaError_t launch_subsplit_reduce(const float* sub_o, const float* sub_lse, int nsub, int n,
+                                   float* part_o, float* part_lse, int B, int T, int Hq, int D,
+                                   cudaStream_t stream);
 
 // ---- error message of the calling thread (star_last_error) -------------------
 void set_last_error(const char* msg);

@@ -49,6 +49,43 @@ def test_version_and_empty_error(lib):
     assert b"sm_100a" in lib.star_version()
 
 
+def _subsplits(B, Hq, Hkv, T, L, b):
+    """Sub-splits per block of a query chunk: fill one wave of 148 CTAs with
+    (split, query tile, head group) items, equal 128-key multiples, at most 4."""
+    if L % b:
+        return 1
+    n = L // b
+    g = Hq // Hkv
+    hpc = 2 if g % 2 == 0 else 1
+    per_split = B * Hkv * (g // hpc) * -(-T // 128)
+    if (n + 1) * per_split >= 148:
+        return 1
+    nsub = min(4, (148 - per_split) // (n * per_split))
+    while nsub > 1 and b % (nsub * 128):
+        nsub -= 1
+    return max(1, nsub)
+
+
+def _chunk_scratch(B, T, Hq, Hkv, D, Lcap, b):
+    up = lambda x: -(-x // 256) * 256  # noqa: E731
+    best = 0
+    for n in range(1, Lcap // b + 1):
+        ns = _subsplits(B, Hq, Hkv, T, n * b, b)
+        if ns > 1:
+            rows = B * Hq * (n * ns + 1) * T
+            best = max(best, up(rows * D * 4) + up(rows * 4))
+    return best
+
+
+def test_query_chunk_subsplit_rule():
+    # llama8b-16k query chunk: 80 items -> 2 sub-splits per block, 144 items
+    assert _subsplits(1, 32, 8, 128, 16384, 4096) == 2
+    # enough items already (llama70b-128k, 256 tokens): no cut
+    assert _subsplits(1, 64, 8, 256, 131072, 32768) == 1
+    # a ragged context is never cut
+    assert _subsplits(1, 32, 8, 128, 16000, 4096) == 1
+
+
 def test_workspace_sizes(lib):
     # Phase 1: status header + rotated Q (bf16)
     assert lib.star_phase1_workspace_bytes(1, 2048, 4, 64) == 256 + 2048 * 4 * 64 * 2
@@ -58,7 +95,7 @@ def test_workspace_sizes(lib):
     chunk = lib.star_phase2_workspace_bytes(1, 128, 32, 8, 128, 16384 + 192, 4096)
     splits = -(-(16384 + 192) // 4096) + 1
     header = 256 + (-(-(8 * splits * 4) // 256)) * 256 + 256
-    assert chunk == header + 128 * 32 * 128 * 2
+    assert chunk == header + 128 * 32 * 128 * 2 + _chunk_scratch(1, 128, 32, 8, 128, 16384 + 192, 4096)
     # decode path adds chunk scratch
     dec = lib.star_phase2_workspace_bytes(1, 1, 32, 8, 128, 16384 + 192, 4096)
     assert dec > 256 + 32 * 128 * 2
