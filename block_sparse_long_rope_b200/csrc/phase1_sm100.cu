@@ -75,9 +75,10 @@ __device__ __forceinline__ float exp2_poly(float x) {
 
 // One pair of keys in kPolyEvery is exponentiated on the FMA pipe instead of
 // the MUFU unit (0 = never). The MUFU exp2 work of a KV tile equals the
-// tensor cores' MMA time at D = 128, but on B200 every tried fraction (1/8,
-// 1/4 of the pairs) cost more issue slots than it saved: 16K-context Phase 1
-// ran at 1104 / 1074 / 1012 TFLOP/s for none / 1/8 / 1/4.
+// tensor cores' MMA time at D = 128, but on B200 every tried fraction cost
+// more than it saved: 16K-context Phase 1 ran at 1104 / 1074 / 1012 TFLOP/s
+// for none / 1/8 / 1/4 of the pairs with this scalar polynomial, and at 1113
+// against 1057-1060 for 1/4 and 1/3 with a packed (f32x2) degree-3 one.
 constexpr int kPolyEvery = 0;
 
 constexpr int kAttnThreads = 320;
