@@ -50,3 +50,12 @@ def test_job_value_is_weak_scaling_throughput():
     # 2 ranks x 16384 tokens each, slowest step 4 ms
     assert bench.job_value(16384, 2, 4.0) == pytest.approx(2 * 16384 / 0.004)
     assert bench.max_over_ranks([1.0, 2.0], None, 1) == [1.0, 2.0]
+
+
+def test_peak_follows_the_sampled_clocks():
+    peaks = {"bf16_tflops": 1669.5, "bf16_tflops_sustained": 1411.1}
+    # full clocks: the burst GEMM figure; power cap engaged: the sustained one
+    assert bench.pick_bf16_peak(peaks, "measured", {"reasons": []})[0] == 1669.5
+    p, src = bench.pick_bf16_peak(peaks, "measured", {"reasons": ["sw_power_cap"]})
+    assert p == 1411.1 and "sustained" in src
+    assert bench.pick_bf16_peak({"bf16_tflops": 1590.0}, "fallback", None)[0] == 1590.0
