@@ -206,6 +206,27 @@ def omp_threads():
 
 
 # --------------------------------------------------------------------------- star arm
+def pack_calls(calls, device=None, pin=False):
+    """The Phase-2 inputs of a step (every call's q, k, v) laid out back to
+    back in one bf16 buffer, so a step uploads them with one copy: returns
+    (buffer, calls whose q, k, v are views into it). Every tensor holds a
+    multiple of 8 elements, so each view starts 16-byte aligned."""
+    import torch
+
+    sizes = [x.numel() for c in calls for x in c[:3]]
+    buf = torch.empty(sum(sizes), dtype=torch.bfloat16, device=device)
+    if pin:
+        buf = buf.pin_memory()
+    out, off = [], 0
+    for c in calls:
+        views = []
+        for x in c[:3]:
+            views.append(buf[off:off + x.numel()].view(x.shape))
+            off += x.numel()
+        out.append(tuple(views) + (c[3],))
+    return buf, out
+
+
 def run_star(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -302,12 +323,17 @@ def run_star(args, w, rank, world, local_rank):
     # compute of step i and the read-back of step i-1. Two layers (caches,
     # outputs) and two device input sets alternate, so no step waits on a
     # buffer another step still uses except through the events below.
+    # The new tokens of all the step's calls sit back to back in one pinned
+    # staging buffer (as a serving loop would batch them), so the upload is
+    # one copy for them plus one per context tensor: at 55 GB/s over the
+    # host link, ~200 separate small copies cost about a millisecond a step.
     host_ctx = [t.cpu().pin_memory() for t in ctx]
-    host_calls = [tuple(x.cpu().pin_memory() for x in c[:3]) + (c[3],) for c in calls]
+    host_pack, host_calls = pack_calls(calls, pin=True)
+    for hc, c in zip(host_calls, calls):
+        for h, x in zip(hc[:3], c[:3]):
+            h.copy_(x)
     layers2 = [layer, StarLayer(w, device=dev)]
-    dev_sets = [([torch.empty_like(t) for t in ctx],
-                 [tuple(torch.empty_like(x) for x in c[:3]) + (c[3],) for c in calls])
-                for _ in range(2)]
+    dev_sets = [([torch.empty_like(t) for t in ctx], pack_calls(calls, device=dev)) for _ in range(2)]
     # the step's result read back is the last generated token's attention
     # output; the Phase-1 output stays on the device (a decoder's next layer
     # consumes it there)
@@ -321,7 +347,7 @@ def run_star(args, w, rank, world, local_rank):
     ev_down = [torch.cuda.Event() for _ in range(2)]
 
     def compute(k):
-        lay, (dctx, dcalls) = layers2[k], dev_sets[k]
+        lay, (dctx, (_, dcalls)) = layers2[k], dev_sets[k]
         lay.encode(*dctx)
         out = None
         for (q2, k2, v2, tail) in dcalls:
@@ -332,14 +358,12 @@ def run_star(args, w, rank, world, local_rank):
 
     def e2e_step(i):
         k = i % 2
-        lay, (dctx, dcalls) = layers2[k], dev_sets[k]
+        lay, (dctx, (dpack, _)) = layers2[k], dev_sets[k]
         s_up.wait_event(ev_comp[k])        # step i-2 no longer reads these inputs
         with torch.cuda.stream(s_up):
             for d, h in zip(dctx, host_ctx):
                 d.copy_(h, non_blocking=True)
-            for dc, hc in zip(dcalls, host_calls):
-                for d, h in zip(dc[:3], hc[:3]):
-                    d.copy_(h, non_blocking=True)
+            dpack.copy_(host_pack, non_blocking=True)
             ev_up[k].record(s_up)
         s_comp.wait_event(ev_up[k])
         s_comp.wait_event(ev_down[k])      # step i-2's outputs have been read back
@@ -617,9 +641,12 @@ def run_sharded(args, w, rank, world, local_rank):
 
     # end to end: this rank's shard and the anchor rows from pinned host memory
     host_ctx = [t.cpu().pin_memory() for t in ctx + anchor]
-    host_calls = [tuple(x.cpu().pin_memory() for x in c[:3]) + (c[3],) for c in calls]
+    host_pack, host_calls = pack_calls(calls, pin=True)  # one copy for all new tokens
+    for hc, c in zip(host_calls, calls):
+        for h, x in zip(hc[:3], c[:3]):
+            h.copy_(x)
     dev_ctx = [torch.empty_like(t) for t in ctx + anchor]
-    dev_calls = [tuple(torch.empty_like(x) for x in c[:3]) + (c[3],) for c in calls]
+    dev_pack, dev_calls = pack_calls(calls, device=dev)
     host_dec = torch.empty((w.B, 1, w.Hq, w.D), dtype=torch.bfloat16).pin_memory()
     h2d = sum(t.numel() * t.element_size() for t in host_ctx) + \
         sum(x.numel() * x.element_size() for c in host_calls for x in c[:3])
@@ -628,9 +655,7 @@ def run_sharded(args, w, rank, world, local_rank):
     def e2e_step():
         for d, h in zip(dev_ctx, host_ctx):
             d.copy_(h, non_blocking=True)
-        for dc, hc in zip(dev_calls, host_calls):
-            for d, h in zip(dc[:3], hc[:3]):
-                d.copy_(h, non_blocking=True)
+        dev_pack.copy_(host_pack, non_blocking=True)
         layer.encode(*dev_ctx[:3], anchor_k=dev_ctx[3], anchor_v=dev_ctx[4])
         out = None
         for (q2, k2, v2, tail) in dev_calls:

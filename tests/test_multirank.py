@@ -59,3 +59,32 @@ def test_peak_follows_the_sampled_clocks():
     p, src = bench.pick_bf16_peak(peaks, "measured", {"reasons": ["sw_power_cap"]})
     assert p == 1411.1 and "sustained" in src
     assert bench.pick_bf16_peak({"bf16_tflops": 1590.0}, "fallback", None)[0] == 1590.0
+
+
+def test_packed_phase2_inputs_alias_one_aligned_buffer():
+    from block_sparse_long_rope_b200.configs import Workload
+    from block_sparse_long_rope_b200.pipeline import phase2_calls
+
+    w = Workload(index=70, name="pack-test", B=2, Hq=8, Hkv=2, D=64, theta=1e4, L=512,
+                 block_len=128, anchor_len=128, Tq=5, Tdec=3)
+    g = torch.Generator().manual_seed(5)
+    new = [torch.randn(w.B, w.Tq + w.Tdec, h, w.D, generator=g).to(torch.bfloat16)
+           for h in (w.Hq, w.Hkv, w.Hkv)]
+    calls = phase2_calls(w, *new)
+    buf, packed = bench.pack_calls(calls)
+    assert buf.numel() == sum(x.numel() for c in calls for x in c[:3])
+    base = buf.data_ptr()
+    for pc, c in zip(packed, calls):
+        assert pc[3] == c[3]
+        for v, x in zip(pc[:3], c[:3]):
+            assert v.shape == x.shape and v.is_contiguous()
+            assert base <= v.data_ptr() < base + buf.numel() * 2
+            assert (v.data_ptr() - base) % 16 == 0
+            v.copy_(x)
+    # one copy of the buffer carries every call's inputs
+    buf2 = buf.clone()
+    off = 0
+    for c in calls:
+        for x in c[:3]:
+            assert torch.equal(buf2[off:off + x.numel()].view(x.shape), x)
+            off += x.numel()
