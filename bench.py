@@ -205,6 +205,21 @@ def omp_threads():
     return int(v) if v else (os.cpu_count() or 1)
 
 
+def host_cpu():
+    """The host's CPU model (first 'model name' of /proc/cpuinfo) and its
+    logical core count, recorded beside the CPU baseline."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "host_cores": os.cpu_count()}
+
+
 # --------------------------------------------------------------------------- star arm
 def pack_calls(calls, device=None, pin=False):
     """The Phase-2 inputs of a step (every call's q, k, v) laid out back to
@@ -573,7 +588,8 @@ def run_star(args, w, rank, world, local_rank):
         est_step, sample, spent = oracle_sample(w, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": round(w.B * w.L / est_step, 3), "unit": "tok/s",
                                 "cores": omp_threads(), "kind": "oracle", "sample": sample,
-                                "seconds_spent": round(spent, 2), "extrapolated": True}
+                                "seconds_spent": round(spent, 2), "extrapolated": True,
+                                **host_cpu()}
     return line
 
 
@@ -725,7 +741,8 @@ def run_sharded(args, w, rank, world, local_rank):
         est_step, sample, spent = oracle_sample(w, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": round(w.B * w.L / est_step, 3), "unit": "tok/s",
                                 "cores": omp_threads(), "kind": "oracle", "sample": sample,
-                                "seconds_spent": round(spent, 2), "extrapolated": True}
+                                "seconds_spent": round(spent, 2), "extrapolated": True,
+                                **host_cpu()}
     return line
 
 
@@ -753,7 +770,8 @@ def run_reference(args, w, rank):
         "config": {"workload": w.name, "B": w.B, "L": w.L, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
                    "block_len": w.block_len, "anchor_len": w.anchor_len},
         "cpu_baseline": {"value": round(value, 3), "unit": "tok/s", "cores": omp_threads(),
-                         "kind": "oracle", "sample": sample, "extrapolated": True},
+                         "kind": "oracle", "sample": sample, "extrapolated": True,
+                         **host_cpu()},
         "e2e": {"value": round(value, 3), "unit": "tok/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "wall_s": round(wall, 2),

@@ -88,3 +88,9 @@ def test_packed_phase2_inputs_alias_one_aligned_buffer():
         for x in c[:3]:
             assert torch.equal(buf2[off:off + x.numel()].view(x.shape), x)
             off += x.numel()
+
+
+def test_host_cpu_reports_model_and_cores():
+    info = bench.host_cpu()
+    assert info["host_cores"] == os.cpu_count()
+    assert isinstance(info["cpu_model"], str) and info["cpu_model"]
