@@ -155,3 +155,19 @@ def test_phase2_items_cover_each_split_row_once_with_exactly_its_keys(lib, geo):
                      for u in range(nsub)]
             assert parts[0][0] == blk * b and parts[-1][1] == min((blk + 1) * b, L)
             assert all(p[1] == q[0] for p, q in zip(parts, parts[1:]))
+
+
+def test_rope_unit_index_by_multiply_high_is_exact_for_every_head_count():
+    """The RoPE kernel splits a unit u = t * per_tok + rem (token, then head and
+    16-byte chunk) with one multiply-high by magic = floor((2^32 - 1) / per_tok)
+    + 1 instead of a division; per_tok = H * D / 16 for H <= 2048 heads and a
+    CTA covers 8 tokens, so u < 8 * per_tok. Checked here against integer
+    division for every head count and both head sizes, every u."""
+    for D in (64, 128):
+        cpr = D // 16
+        for H in range(1, 2049):
+            d = H * cpr
+            magic = (0xFFFFFFFF // d) + 1
+            u = np.arange(8 * d, dtype=np.uint64)
+            t = (u * np.uint64(magic)) >> np.uint64(32)
+            assert np.array_equal(t, u // np.uint64(d)), (D, H)
