@@ -133,3 +133,76 @@ def test_rounded_qk_mode_equals_brute_on_rounded_inputs():
     # happens here, so agreement is to fp64 rounding of the attention itself
     np.testing.assert_allclose(o[0], ro, rtol=0, atol=1e-12)
     np.testing.assert_allclose(lse[0], rl, rtol=0, atol=1e-12)
+
+
+def _edge_rows(L, b):
+    """Rows at block starts and ends, 128-row tile edges, and a few inside."""
+    rows = set()
+    for s in range(0, L, b):
+        for r in (s, s + 1, s + b - 1, s + b - 2):
+            if 0 <= r < L:
+                rows.add(r)
+        for t in range(s, min(s + b, L), 128):
+            for r in (t - 1, t, t + 127):
+                if s <= r < min(s + b, L):
+                    rows.add(r)
+    rows.add(L - 1)
+    return sorted(rows)
+
+
+@pytest.mark.parametrize("B,L,b,a,g,Hkv", [(2, 300, 128, 128, 1, 2), (2, 1000, 300, 200, 4, 2),
+                                           (3, 520, 256, 100, 8, 1), (2, 640, 640, 640, 4, 1),
+                                           (2, 777, 129, 0, 8, 2)])
+def test_selected_rows_equal_full_tensor_rows(B, L, b, a, g, Hkv):
+    """phase1_rows_selected (queries passed one by one, as the full-size
+    checks do) gives exactly the bits of phase1_rows on the whole Q tensor,
+    for random (batch, head, row) picks and rows at block and tile edges."""
+    Hq, D, theta = g * Hkv, 16, 5e5
+    gen = torch.Generator().manual_seed(B * 1000 + L + b + a + g)
+    q = torch.randn(B, L, Hq, D, generator=gen).to(torch.bfloat16)
+    k = torch.randn(B, L, Hkv, D, generator=gen).to(torch.bfloat16)
+    v = torch.randn(B, L, Hkv, D, generator=gen).to(torch.bfloat16)
+    rng = np.random.default_rng(L + b)
+    edge = np.array(_edge_rows(L, b))
+    nr = 60
+    rows = np.concatenate([edge, rng.integers(0, L, size=nr)])
+    qb = rng.integers(0, B, size=rows.size)
+    qh = rng.integers(0, Hq, size=rows.size)
+    perm = rng.permutation(rows.size)  # the selection's order is arbitrary
+    rows, qb, qh = rows[perm], qb[perm], qh[perm]
+    q_sel = q[torch.as_tensor(qb), torch.as_tensor(rows), torch.as_tensor(qh)]  # [nq, D]
+    for round_qk in (True, False):
+        o_ref, l_ref, n_ref = orc.phase1_rows(q, k, v, b, a, theta, qb, qh, rows, round_qk)
+        o, lse, nvis = orc.phase1_rows_selected(q_sel, k, v, b, a, theta, qb, qh, rows, Hq,
+                                                round_qk)
+        np.testing.assert_array_equal(o, o_ref)
+        np.testing.assert_array_equal(lse, l_ref)
+        np.testing.assert_array_equal(nvis, n_ref)
+
+
+@pytest.mark.parametrize("L,b,a,g", [(48, 12, 12, 1), (50, 16, 5, 4), (40, 40, 40, 8),
+                                     (45, 10, 0, 2)])
+def test_selected_rows_match_dense_mask_brute_force(L, b, a, g):
+    """phase1_rows_selected against the dense-mask brute force directly, on
+    every row of two sequences, heads of every GQA group, rows given in
+    reverse order."""
+    B, Hkv, D, theta = 2, 2, 8, 1e4
+    Hq = g * Hkv
+    gen = torch.Generator().manual_seed(400 + L + b + a + g)
+    q = torch.randn(B, L, Hq, D, generator=gen).to(torch.bfloat16)
+    k = torch.randn(B, L, Hkv, D, generator=gen).to(torch.bfloat16)
+    v = torch.randn(B, L, Hkv, D, generator=gen).to(torch.bfloat16)
+    bb, hh, rr = np.meshgrid(np.arange(B), np.arange(Hq), np.arange(L)[::-1], indexing="ij")
+    qb, qh, qr = bb.ravel(), hh.ravel(), rr.ravel()
+    q_sel = q[torch.as_tensor(qb), torch.as_tensor(qr), torch.as_tensor(qh)]
+    o, lse, nvis = orc.phase1_rows_selected(q_sel, k, v, b, a, theta, qb, qh, qr, Hq,
+                                            round_qk=False)
+    M = brute.phase1_mask(L, b, a)
+    for bi in range(B):
+        qrot = brute.rope_complex(q[bi].double().numpy(), np.arange(L), theta)
+        krot = brute.rope_complex(k[bi].double().numpy(), np.arange(L), theta)
+        ro, rl = brute.phase1_dense(qrot, krot, v[bi].double().numpy(), b, a)
+        sel = qb == bi
+        np.testing.assert_allclose(o[sel], ro[qr[sel], qh[sel]], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(lse[sel], rl[qh[sel], qr[sel]], rtol=0, atol=1e-12)
+        np.testing.assert_array_equal(nvis[sel], M.sum(1)[qr[sel]])
