@@ -33,6 +33,7 @@ EXPORTS = (
     "star_phase2_workspace_bytes",
     "star_phase2_partial",
     "star_phase2_decode_static",
+    "star_phase2_decode_static_status",
     "star_phase2_attend",
     "star_lse_merge",
     "star_rmsnorm",
@@ -106,6 +107,8 @@ def load(path: str = LIB_PATH):
         lib.star_phase2_decode_static.restype = _I
         lib.star_phase2_decode_static.argtypes = [_P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P,
                                                   _IP, _I, _I, _I, _I, _D, _P]
+        lib.star_phase2_decode_static_status.restype = _I
+        lib.star_phase2_decode_static_status.argtypes = [_P]
         lib.star_phase2_attend.restype = _I
         lib.star_phase2_attend.argtypes = [_P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _P, _P, _P, _P,
                                            _IP, _I, _I, _I, _I, _D, _P, _SZ, _P]

@@ -10,6 +10,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 #include <string>
 
@@ -195,13 +196,31 @@ namespace star {
 // Sets the calling thread's message for star_last_error (used by entry points
 // defined in other files of the library).
 void set_last_error(const char* msg) { g_err = msg; }
+
+cudaError_t set_smem_attr_once(const void* fn, int slot, int dev, size_t bytes) {
+  static std::atomic<bool> done[kAttrSlots][64];
+  static std::mutex mu;
+  const bool cacheable = slot >= 0 && slot < kAttrSlots && dev >= 0 && dev < 64;
+  if (cacheable && done[slot][dev].load(std::memory_order_acquire)) return cudaSuccess;
+  std::lock_guard<std::mutex> lk(mu);
+  if (cacheable && done[slot][dev].load(std::memory_order_relaxed)) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(bytes));
+  if (e == cudaSuccess && cacheable) done[slot][dev].store(true, std::memory_order_release);
+  return e;
+}
 }  // namespace star
 
 extern "C" {
 
 const char* star_last_error(void) { return g_err.c_str(); }
 
-const char* star_version(void) { return "star-b200 0.1 (sm_100a)"; }
+#ifndef STAR_BUILD_DIGEST
+#define STAR_BUILD_DIGEST "unknown"
+#endif
+// The build digest (sources, headers, flags) ends the string, so a caller can
+// check that the library it loaded was built from the sources it has.
+const char* star_version(void) { return "star-b200 0.2 (sm_100a) build " STAR_BUILD_DIGEST; }
 
 star_status star_rope(const void* x, const int64_t x_stride[3], void* y, const int64_t y_stride[3],
                       const int32_t* pos, int64_t pos0, int B, int S, int H, int D, double theta,

@@ -15,11 +15,12 @@
 //    call made with that device current (cudaGetSymbolAddress). Make that
 //    first call before any stream capture.
 //  * Every call on a device shares the one array and it keeps the previous
-//    call's contents. The status word and the per-split chunk counters at
-//    its start are cleared by every call; everything else is fully
-//    rewritten before it is read. Calls whose work
-//    overlaps on the GPU (different streams, or host threads without
-//    ordering) race on the array: serialise them.
+//    call's contents. The per-split chunk counters are cleared by every call;
+//    everything else is fully rewritten before it is read, except the status
+//    word: device errors (a bounded wait that gave up) are ORed into it and
+//    stay there until star_phase2_decode_static_status reads and clears it.
+//    Calls whose work overlaps on the GPU (different streams, or host
+//    threads without ordering) race on the array: serialise them.
 //  * Sizes that cannot fit are rejected with STAR_ERR_INVALID_ARG before
 //    anything is enqueued. Nothing here allocates.
 #include <cuda.h>
@@ -200,8 +201,10 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
 
   cudaStream_t stream = static_cast<cudaStream_t>(cuda_stream);
   unsigned char* ws = static_cast<unsigned char*>(base);
-  cudaError_t e = cudaMemsetAsync(ws, 0, zero_bytes, stream);
-  if (e != cudaSuccess) return fail_static(STAR_ERR_CUDA, "status reset: %s", cudaGetErrorString(e));
+  // the counters start at zero; the status block before them is left alone
+  // (sticky until star_phase2_decode_static_status)
+  cudaError_t e = cudaMemsetAsync(ws + star::kStatusBytes, 0, zero_bytes - star::kStatusBytes, stream);
+  if (e != cudaSuccess) return fail_static(STAR_ERR_CUDA, "counter reset: %s", cudaGetErrorString(e));
 
   star::DecodeParams dp;
   memset(&dp, 0, sizeof dp);
@@ -246,6 +249,28 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
   e = star::launch_decode(dp, D, stream);
   if (e != cudaSuccess) return fail_static(STAR_ERR_CUDA, "decode launch: %s", cudaGetErrorString(e));
   if (nsplit_out) *nsplit_out = n + 1;
+  return STAR_OK;
+}
+
+star_status star_phase2_decode_static_status(void* cuda_stream) {
+  star::set_last_error("");
+  void* base = nullptr;
+  int sms = 0;
+  star_status st = scratch_address(&base, &sms);
+  if (st != STAR_OK) return st;
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return fail_static(STAR_ERR_CUDA, "stream synchronize: %s", cudaGetErrorString(e));
+  int word = 0;
+  e = cudaMemcpy(&word, base, sizeof word, cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return fail_static(STAR_ERR_CUDA, "status read: %s", cudaGetErrorString(e));
+  if (word != 0) {
+    e = cudaMemset(base, 0, sizeof word);
+    if (e != cudaSuccess) return fail_static(STAR_ERR_CUDA, "status clear: %s", cudaGetErrorString(e));
+  }
+  if (word & star::kDevTimeout)
+    return fail_static(STAR_ERR_DEVICE_TIMEOUT, "a decode kernel's bounded wait gave up (status 0x%x)", word);
+  if (word & star::kDevBounds)
+    return fail_static(STAR_ERR_DEVICE_BOUNDS, "a decode kernel found an index outside its buffer (status 0x%x)", word);
   return STAR_OK;
 }
 

@@ -57,30 +57,6 @@ struct AttnCfg {
   static constexpr uint32_t kTmemCols = 512;
 };
 
-// 2^x on the FMA pipe: x = n + f with n = round(x), f in [-1/2, 1/2];
-// 2^f by a degree-4 polynomial (relative error < 3e-6, fitted by
-// fit_exp2_poly.py), 2^n added to the exponent bits. x is clamped at -126
-// (the result is then < 2^-125, i.e. zero for the softmax).
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;  // 1.5 * 2^23: round(x) lands in the low mantissa bits
-  const float f = x - (t - 12582912.f);
-  const int n = __float_as_int(t) - 0x4B400000;
-  float p = fmaf(9.560510516e-03f, f, 5.591703951e-02f);
-  p = fmaf(p, f, 2.402498126e-01f);
-  p = fmaf(p, f, 6.931219697e-01f);
-  p = fmaf(p, f, 9.999991655e-01f);
-  return __int_as_float(__float_as_int(p) + (n << 23));
-}
-
-// One pair of keys in kPolyEvery is exponentiated on the FMA pipe instead of
-// the MUFU unit (0 = never). The MUFU exp2 work of a KV tile equals the
-// tensor cores' MMA time at D = 128, but on B200 every tried fraction cost
-// more than it saved: 16K-context Phase 1 ran at 1104 / 1074 / 1012 TFLOP/s
-// for none / 1/8 / 1/4 of the pairs with this scalar polynomial, and at 1113
-// against 1057-1060 for 1/4 and 1/3 with a packed (f32x2) degree-3 one.
-constexpr int kPolyEvery = 0;
-
 constexpr int kAttnThreads = 320;
 constexpr uint64_t kDrainNs = 100000000ull;  // 100 ms
 
@@ -358,10 +334,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
       }
       const float ref = (m_run == -INFINITY) ? 0.f : m_run * c;
       // x = s * c - ref for two keys at once (fma.rn.f32x2), exp2 on the MUFU
-      // unit except every kPolyEvery-th pair (FMA pipe), row sums in four
-      // packed accumulators. P (bf16 pairs) goes back over the first 64
-      // columns of S, 32 keys at a time; S columns 16q.. are already
-      // consumed when quarter q is written.
+      // unit, row sums in four packed accumulators. P (bf16 pairs) goes back
+      // over the first 64 columns of S, 32 keys at a time; S columns 16q..
+      // are already consumed when quarter q is written.
       const uint64_t cc = f2_pack(c, c), nref = f2_pack(-ref, -ref);
       uint64_t ls[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -372,16 +347,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
           float x0, x1;
           f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[q][2 * j]), __uint_as_float(sr[q][2 * j + 1])),
                            cc, nref), x0, x1);
-          float p0 = 0.f, p1 = 0.f;
-          bool on_fma = false;
-          if constexpr (kPolyEvery > 0) on_fma = (j % (kPolyEvery > 0 ? kPolyEvery : 1)) == kPolyEvery - 1;
-          if (on_fma) {
-            p0 = exp2_poly(x0);
-            p1 = exp2_poly(x1);
-          } else {
-            p0 = ex2_approx(x0);
-            p1 = ex2_approx(x1);
-          }
+          const float p0 = ex2_approx(x0), p1 = ex2_approx(x1);
           ls[j & 3] = f2_add(ls[j & 3], f2_pack(p0, p1));
           pk[j] = pack_bf16x2(p0, p1);
         }
@@ -463,24 +429,13 @@ cudaError_t launch_attn(const AttnParams& p, int D, cudaStream_t stream) {
   const size_t smem = attn_smem_bytes(D);
   int dev = 0;
   cudaGetDevice(&dev);
-  static bool attr128[64] = {}, attr64[64] = {};
-  if (D == 128) {
-    if (dev < 64 && !attr128[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(attn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      attr128[dev] = true;
-    }
+  cudaError_t ea = set_smem_attr_once(D == 128 ? (const void*)attn_kernel<128> : (const void*)attn_kernel<64>,
+                                      D == 128 ? 3 : 2, dev, smem);
+  if (ea != cudaSuccess) return ea;
+  if (D == 128)
     attn_kernel<128><<<p.num_items, kAttnThreads, smem, stream>>>(p);
-  } else {
-    if (dev < 64 && !attr64[dev]) {
-      cudaError_t e = cudaFuncSetAttribute(attn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           static_cast<int>(smem));
-      if (e != cudaSuccess) return e;
-      attr64[dev] = true;
-    }
+  else
     attn_kernel<64><<<p.num_items, kAttnThreads, smem, stream>>>(p);
-  }
   return cudaGetLastError();
 }
 

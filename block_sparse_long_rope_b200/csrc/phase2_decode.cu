@@ -345,10 +345,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
       prefetch_tmap(&p.tmK);
       prefetch_tmap(&p.tmV);
     }
-    // Only a decode kernel starts this one before it ends (no other kernel of
-    // the library triggers its dependents), and a decode kernel never writes
-    // cache rows [0, L) or q: tiles of those rows are loaded at once; the
-    // tail rows (appended by the previous step) and the append wait for the
+    // The previous kernel in the stream may still be running (programmatic
+    // dependent launch). Cache rows [0, L) are written only by Phase 1,
+    // whose kernels never start a dependent early and are always followed by
+    // another kernel, so tiles of those rows are loaded at once; the tail
+    // rows (appended by the previous step) and the append wait for the
     // previous kernel's end.
     bool waited = false;
     const int row0 = p.L + p.tail_len;  // cache row of new token 0
@@ -429,6 +430,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
     const float c = p.scale_log2;
     uint32_t qf[kKSteps][4];
     int q_bh = -1;
+    bool q_waited = false;
     int gt = 0;  // tiles consumed over all units of this CTA
     for (int u = u_begin; u < u_end; ++u) {
       const int bh = u / p.chunks_per_head;
@@ -458,6 +460,14 @@ __global__ void __launch_bounds__(kDecThreads, 2) decode_kernel(const __grid_con
             rope_angle(static_cast<long long>(p.q_pos0) + t0 + e / (D / 2),
                        p.inv_freq[e % (D / 2)], &tcos[e], &tsin[e]);
           consumer_sync();
+          // q may be written by the kernel just before this one (a projection,
+          // or a caller's own kernel that starts its dependents early): read
+          // it only after that kernel has ended. The cos/sin table above
+          // depends on positions only and is built before the wait.
+          if (!q_waited) {
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            q_waited = true;
+          }
           for (int e = threadIdx.x; e < tn * g * (D / 2); e += kConsumers) {
             const int rl = e / (D / 2), i = e % (D / 2);
             const int tl = rl / g, rho = t0 * g + rl;
@@ -656,15 +666,9 @@ cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t stream) {
   const size_t smem = decode_smem_bytes(D);
   int dev = 0;
   cudaGetDevice(&dev);
-  static bool attr128[64] = {}, attr64[64] = {};
-  bool* attr = (D == 128) ? attr128 : attr64;
-  if (dev >= 64 || !attr[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(D == 128 ? decode_kernel<128> : decode_kernel<64>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    if (dev < 64) attr[dev] = true;
-  }
+  cudaError_t ea = set_smem_attr_once(D == 128 ? (const void*)decode_kernel<128> : (const void*)decode_kernel<64>,
+                                      D == 128 ? 1 : 0, dev, smem);
+  if (ea != cudaSuccess) return ea;
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = imin(units, 2 * sms);  // persistent: two CTAs per SM

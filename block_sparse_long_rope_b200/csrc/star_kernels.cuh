@@ -123,6 +123,14 @@ cudaError_t launch_subsplit_reduce(const float* sub_o, const float* sub_lse, int
 // ---- error message of the calling thread (star_last_error) -------------------
 void set_last_error(const char* msg);
 
+// ---- per-device launch set-up ---------------------------------------------------
+// Raises kernel `fn`'s dynamic shared-memory limit to `bytes` on device `dev`
+// the first time it is asked for that (slot, device); later calls return at
+// once. Safe to call from several host threads. slot < kAttrSlots names the
+// kernel (one slot per kernel instantiation).
+constexpr int kAttrSlots = 8;
+cudaError_t set_smem_attr_once(const void* fn, int slot, int dev, size_t bytes);
+
 // ---- debug: device-evaluated index math --------------------------------------
 cudaError_t launch_debug_index(int L, int b, int a, int32_t* blk, int32_t* pos, int32_t* ranges,
                                cudaStream_t stream);

@@ -213,6 +213,12 @@ def star_phase2_decode_static(q, k, v, k_cache, v_cache, L, block_len, tail_len,
     return ns.value
 
 
+def star_phase2_decode_static_status(stream=None):
+    """Reads and clears the device-error word of star_phase2_decode_static
+    (synchronises the stream); raises StarError on a device error."""
+    _abi.check(_abi.load().star_phase2_decode_static_status(_stream(stream)))
+
+
 def star_lse_merge(part_o, part_lse, o, lse=None, stream=None):
     """Exact merge: part_o[B,Hq,S,T,D], part_lse[B,Hq,S,T] -> o[B,T,Hq,D] bf16, lse[B,Hq,T]."""
     B, Hq, S, T, D = part_o.shape

@@ -47,10 +47,12 @@
  *     Lcap and block_len; before any other reuse it must be zero-filled
  *     again. No call resets the workspace, so consecutive decode kernels run
  *     back to back: the decode kernel is launched as a programmatic dependent
- *     launch. Only a decode kernel can start it early, so it streams cache
- *     rows [0, L) and reads q before that kernel has finished, and waits for
- *     it before touching the tail rows and before its first write.
- *     Consecutive decode calls on one cache must therefore keep the context
+ *     launch and may start while the previous kernel in the stream drains.
+ *     It streams cache rows [0, L) at once and waits for that kernel to end
+ *     before it reads q, k or v, touches the tail rows, or writes anything.
+ *     Cache rows [0, L) must therefore not be written by the kernel launched
+ *     just before a decode call (Phase 1 never is: its last kernel only reads
+ *     the cache), and consecutive decode calls on one cache keep the context
  *     length L and grow only the tail. This is how Phase 2 proceeds: the
  *     context is fixed after Phase 1.
  */
@@ -77,7 +79,8 @@ typedef enum {
  * The pointer stays valid until the next call on the same thread. */
 const char* star_last_error(void);
 
-/* Library version string. */
+/* Library version string; it ends with the digest of the sources, headers and
+ * build flags the library was built from. */
 const char* star_version(void);
 
 /*
@@ -296,9 +299,11 @@ star_status star_lse_merge_ranks(const float* part_o, const float* part_lse, int
  *     with that device current; make that first call before any stream
  *     capture.
  *   - All calls on a device share the array, which keeps the previous call's
- *     contents (the status word is cleared by each call; the rest is rewritten
- *     before it is read). Calls whose work overlaps on the GPU race on it:
- *     serialise them (one stream, or explicit ordering).
+ *     contents: each call clears the split counters and rewrites the partials
+ *     before reading them; device errors are ORed into a status word that
+ *     stays set until star_phase2_decode_static_status reads it. Calls whose
+ *     work overlaps on the GPU race on the array: serialise them (one stream,
+ *     or explicit ordering).
  *   - Sizes whose scratch cannot fit 16 MiB even with the largest chunk, or
  *     T * g > 16, return STAR_ERR_INVALID_ARG before anything is enqueued.
  *     Nothing is allocated.
@@ -308,6 +313,21 @@ star_status star_phase2_decode_static(const void* q, const void* k, const void* 
                                       int block_len, int tail_len, float* part_o,
                                       float* part_lse, int* nsplit_out, int B, int Hq, int Hkv,
                                       int D, double theta, void* cuda_stream);
+
+/*
+ * star_phase2_decode_static_status — the device-error read-back of
+ * star_phase2_decode_static, which has no workspace for star_device_status
+ * to read. The pages have no counterpart. Synchronises `cuda_stream`, reads
+ * the status word kept at the start of the current device's static array
+ * (device errors of every star_phase2_decode_static call since the last
+ * read are ORed into it: a bounded wait that gave up, an index outside its
+ * buffer) and clears it. Returns STAR_OK, STAR_ERR_DEVICE_TIMEOUT or
+ * STAR_ERR_DEVICE_BOUNDS (message in star_last_error), or STAR_ERR_CUDA.
+ * After a device error the outputs of the calls since the last read are not
+ * valid. Allocates nothing; the first call on a device looks up the array's
+ * address like star_phase2_decode_static does.
+ */
+star_status star_phase2_decode_static_status(void* cuda_stream);
 
 /*
  * Layers around Star attention in a decoder stack. Star Attention replaces

@@ -49,6 +49,27 @@ def test_version_and_empty_error(lib):
     assert b"sm_100a" in lib.star_version()
 
 
+def test_loaded_library_was_built_from_these_sources(lib):
+    # the build digest (sources, headers, flags) ends the version string
+    assert star_build.loaded_matches_sources(), lib.star_version()
+
+
+def test_phase2_workspace_size_formula(lib):
+    # star_phase2_workspace_bytes(B, T, Hq, Hkv, D, Lcap, block_len): the decode
+    # path's partials depend on Hkv (one 16-row tile per GQA group) and on the
+    # cache capacity (the splits a context of up to Lcap rows can have)
+    up = lambda x: -(-x // 256) * 256  # noqa: E731
+    for B, Hq, Hkv, D, Lcap, b in [(1, 32, 8, 128, 16384 + 192, 4096), (2, 4, 1, 64, 2072, 512),
+                                   (1, 64, 8, 128, 131072 + 384, 32768)]:
+        nsplit_cap = -(-Lcap // b) + 1
+        header = 256 + up(B * Hkv * nsplit_cap * 4) + up(B * Hkv * 4)
+        splits = B * Hkv * nsplit_cap
+        units = max(512, splits) + splits
+        rows = units * 16
+        dec = header + up(B * 1 * Hq * D * 2) + up(rows * D * 4) + up(rows * 4)
+        assert lib.star_phase2_workspace_bytes(B, 1, Hq, Hkv, D, Lcap, b) == dec
+
+
 def _subsplits(B, Hq, Hkv, T, L, b):
     """Sub-splits per block of a query chunk: fill one wave of 148 CTAs with
     (split, query tile, head group) items, equal 128-key multiples, at most 4."""
