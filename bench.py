@@ -8,13 +8,12 @@ merge). Inputs are resident in HBM when the timed region starts.
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl star|reference]
 
 One JSON line on stdout (rank 0). With N > 1 (torchrun, one rank per GPU)
-each rank runs its own independent sequences (weak scaling, no data-path
-collective); the time is the max over ranks.
-
---mode sharded spreads ONE sequence's blocks over the N ranks instead (the
-pages' multi-host form: Phase 1 per shard, Phase 2 with a query broadcast, an
+the default spreads ONE sequence's blocks over the N ranks (the pages'
+multi-host form: Phase 1 per shard, Phase 2 with a query broadcast, an
 all-gather of partials and the merge over NCCL; strong scaling), launched
-eagerly. With N = 1 it runs the same code on a one-rank process group.
+eagerly; the time is the max over ranks. --mode sharded runs the same code
+on a one-rank process group at N = 1. --mode replicas gives every rank its
+own independent sequences instead (weak scaling, no data-path collective).
 """
 import argparse
 import json
@@ -287,47 +286,28 @@ def pack_calls(calls, device=None, pin=False):
 
 def layer_launches(w):
     """Kernels one step of workload w launches: Phase 1 (RoPE + attention),
-    the query chunk (RoPE + attention [+ sub-split reduce] + merge), one
-    decode kernel per token."""
+    the query chunk (RoPE + attention, which reduces and merges in-kernel),
+    one decode kernel per token."""
     chunk = 0
     if w.Tq > 0:
-        g = w.Hq // w.Hkv
-        if w.Tq * g <= 16:
-            chunk = 1  # the decode kernel does it all
-        else:
-            chunk = 3 + (1 if query_chunk_subsplits(w) > 1 else 0)
+        chunk = 1 if w.Tq * (w.Hq // w.Hkv) <= 16 else 2  # the decode kernel does it all
     return 2 + chunk + w.Tdec
 
 
-def query_chunk_subsplits(w):
-    """Sub-splits per context block of the query chunk (the library's rule:
-    fill one wave of 148 CTAs with (split, query tile, head group) items)."""
-    if w.L % w.block_len:
-        return 1
-    n = w.L // w.block_len
-    g = w.Hq // w.Hkv
-    hpc = 2 if g % 2 == 0 else 1
-    per_split = w.B * w.Hkv * (g // hpc) * -(-w.Tq // 128)
-    if (n + 1) * per_split >= 148:
-        return 1
-    nsub = min(4, (148 - per_split) // (n * per_split))
-    while nsub > 1 and w.block_len % (nsub * 128):
-        nsub -= 1
-    return max(1, nsub)
-
-
 def flush_l2(buf):
-    """Overwrites a buffer larger than the 126 MB L2, evicting what it held."""
-    buf.zero_()
+    """Evicts the 126 MB L2 by reading a 256 MiB buffer that is never written
+    (its lines stay clean, so the timed call that follows pays no write-back
+    of dirty lines, as zeroing a buffer would leave it to)."""
+    buf.sum()
 
 
 def cold_decode(layer, call, reps, dev, world):
-    """Mean device time (ms) of one decode call with L2 flushed before each
+    """Mean device time (ms) of one decode call with L2 evicted before each
     repetition (events around the call alone), max over ranks."""
     import torch
 
     q2, k2, v2, tail = call
-    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)  # 256 MiB
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)  # 256 MiB
     for _ in range(2):
         layer.attend(q2, k2, v2, tail)
     torch.cuda.synchronize()
@@ -431,9 +411,9 @@ def side_stack(args, w, dev, world):
 
 def side_phase2(args, w, dev, world, peaks):
     """Phase 2 of workload w after one Phase-1 encode: the query chunk (mean
-    of replays, L2 flushed before each), the decode loop of all Tdec tokens
+    of replays, L2 evicted before each), the decode loop of all Tdec tokens
     as one graph (consecutive steps overlap), and one decode step in
-    isolation with L2 flushed before it."""
+    isolation with L2 evicted before it."""
     import torch
 
     from block_sparse_long_rope_b200 import inputs, star
@@ -446,7 +426,7 @@ def side_phase2(args, w, dev, world, peaks):
     layer.encode(*ctx)
     del ctx
     stream = torch.cuda.current_stream()
-    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)  # 256 MiB
+    flush = torch.ones(64 << 20, dtype=torch.float32, device=dev)  # 256 MiB
     res = {"workload": w.name}
     if w.Tq > 0:
         q2, k2, v2, tail = calls[0]
@@ -681,7 +661,7 @@ def run_star(args, w, rank, world, local_rank):
         star.star_device_status(lay.buf.ws2)
     del layers2[1], dev_sets, replay
 
-    # one decode step in isolation, L2 flushed before it (the cache of the
+    # one decode step in isolation, L2 evicted before it (the cache of the
     # main workload holds every row from the last step)
     cold_main = cold_decode(layer, calls[-1], args.cold_decode_steps, dev, world) \
         if args.cold_decode_steps > 0 and w.Tdec > 0 else None
@@ -748,7 +728,7 @@ def run_star(args, w, rank, world, local_rank):
         phases["phase2_decode"] = d
         if cold_main is not None:
             c = decode_entry(cold_main[0], w.decode_kv_bytes(cold_main[1]), 1, cache,
-                             "one decode call alone, L2 flushed before it (256 MiB written)")
+                             "one decode call alone, L2 evicted before it (256 MiB read)")
             c["tok_s"] = round(w.B / (cold_main[0] / 1e3), 1)
             phases["phase2_decode_cold_step"] = c
     if p2 is not None:
@@ -759,7 +739,7 @@ def run_star(args, w, rank, world, local_rank):
             tf = qc["flops"] / (qc["ms"] / 1e3) / 1e12
             e["query_chunk"] = {"ms": round(qc["ms"], 4), "tokens": qc["tokens"],
                                 "tflops": round(tf, 2), "frac_bf16_peak": round(tf / burst, 4),
-                                "how": "one query-chunk call, L2 flushed before each"}
+                                "how": "one query-chunk call, L2 evicted before each (256 MiB read)"}
         if "decode_loop" in p2:
             dl, dc = p2["decode_loop"], p2["decode_cold"]
             cache2 = w2.decode_kv_bytes(w2.Tq + w2.Tdec - 1)
@@ -768,7 +748,7 @@ def run_star(args, w, rank, world, local_rank):
                                             "overlap and part of the cache stays in L2")
             e["decode_loop"]["tok_s"] = round(w2.B * dl["steps"] / (dl["ms"] / 1e3), 1)
             e["decode_cold_step"] = decode_entry(dc["ms"], dc["bytes"], 1, cache2,
-                                                 "one decode call alone, L2 flushed before it")
+                                                 "one decode call alone, L2 evicted before it (256 MiB read)")
             e["decode_cold_step"]["tok_s"] = round(w2.B / (dc["ms"] / 1e3), 1)
         phases["phase2_" + w2.name.replace("-", "_")] = e
     if pulsar is not None:
@@ -1046,6 +1026,15 @@ def run_reference(args, w, rank):
     }
 
 
+def resolve_mode(mode, world):
+    """The run's multi-GPU mode: as asked, else one sequence's blocks over the
+    ranks when there are several (the pages' hosts: query broadcast, local
+    partials, gather and merge), and a single replica on one GPU."""
+    if mode is not None:
+        return mode
+    return "sharded" if world > 1 else "replicas"
+
+
 def _free_port():
     import socket
 
@@ -1068,16 +1057,17 @@ def main():
                     help="skip the side measurement of Phase 1 with Pulsar's prefix layout")
     ap.add_argument("--stack-layers", type=int, default=2,
                     help="layers of the side measurement of a decoder stack (0 skips it)")
-    ap.add_argument("--mode", default="replicas", choices=["replicas", "sharded"],
+    ap.add_argument("--mode", default=None, choices=["replicas", "sharded"],
                     help="replicas: independent sequences per rank; sharded: one sequence's "
-                         "blocks spread over the ranks")
+                         "blocks spread over the ranks (the pages' deployment; the default "
+                         "with more than one GPU)")
     ap.add_argument("--side-config", default=SIDE_CONFIG,
                     help="workload of the side measurements (Pulsar layout, decoder stack)")
     ap.add_argument("--phase2-config", default=PHASE2_CONFIG,
                     help="workload of the Phase-2 side measurement (query chunk, decode loop "
                          "and cold decode step); '' skips it")
     ap.add_argument("--cold-decode-steps", type=int, default=16,
-                    help="repetitions of the isolated decode step timed with L2 flushed")
+                    help="repetitions of the isolated decode step timed with L2 evicted")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=8.0)
     args = ap.parse_args()
@@ -1094,6 +1084,7 @@ def main():
         if line is not None:
             print(json.dumps(line), flush=True)
         return
+    args.mode = resolve_mode(args.mode, world)
     use_pg = world > 1 or args.mode == "sharded"
     if use_pg:
         import datetime

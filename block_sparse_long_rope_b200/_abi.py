@@ -28,6 +28,7 @@ EXPORTS = (
     "star_phase1_encode",
     "star_phase1_ext_workspace_bytes",
     "star_phase1_encode_ext",
+    "star_phase1_encode_rotated",
     "star_phase2_partial_ext",
     "star_lse_merge_ranks",
     "star_phase2_workspace_bytes",
@@ -38,6 +39,8 @@ EXPORTS = (
     "star_lse_merge",
     "star_rmsnorm",
     "star_linear",
+    "star_linear_rope",
+    "star_linear_rope_workspace_bytes",
     "star_device_status",
     "star_debug_index",
     "star_debug_wait_probe",
@@ -90,6 +93,14 @@ def load(path: str = LIB_PATH):
         lib.star_phase1_encode_ext.restype = _I
         lib.star_phase1_encode_ext.argtypes = [_P, _P, _P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I,
                                                _I, _P, _P, _I, _P, _P, _P, _I, _I, _D, _P, _SZ, _P]
+        lib.star_phase1_encode_rotated.restype = _I
+        lib.star_phase1_encode_rotated.argtypes = [_P, _P, _P, _P, _I, _P, _I, _I, _I, _I, _I, _I,
+                                                   _I, _P, _SZ, _P]
+        lib.star_linear_rope_workspace_bytes.restype = _SZ
+        lib.star_linear_rope_workspace_bytes.argtypes = [_I, _I, _I]
+        lib.star_linear_rope.restype = _I
+        lib.star_linear_rope.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _D, _I, _P,
+                                         _SZ, _P]
         lib.star_phase2_partial_ext.restype = _I
         lib.star_phase2_partial_ext.argtypes = [_P, _P, _P, _I, _P, _P, _I, _I, _I, _I, _I, _I, _I,
                                                 _P, _P, _IP, _I, _I, _I, _I, _D, _P, _SZ, _P]

@@ -24,14 +24,14 @@ LIB = os.path.join(HERE, "libstar.so")
 OBJ_DIR = os.path.join(HERE, "_build")
 
 SOURCES = ["api.cu", "rope.cu", "lse_merge.cu", "phase2_decode.cu", "phase1_sm100.cu", "noalloc.cu",
-           "stack.cu"]
+           "stack.cu", "gemm_sm100.cu"]
 HEADERS = ["star_common.cuh", "star_index.cuh", "star_kernels.cuh", "rope_math.cuh", "star_plan.h"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",
          "-I" + INCLUDE, "-I" + CSRC]
-LINK = ["-lcublasLt"]
+LINK = []
 
 
 def _sha(paths, extra=()):

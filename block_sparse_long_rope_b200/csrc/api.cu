@@ -178,10 +178,19 @@ size_t chunk_scratch_bytes(int B, int T, int Hq, int Hkv, int D, int Lcap, int b
   for (int n = 1; (long long)n * block_len <= Lcap; ++n) {
     const int nsub = chunk_subsplits(B, Hq, Hkv, T, n * block_len, block_len, 1);
     if (nsub <= 1) continue;
-    const size_t rows = (size_t)B * Hq * (n * nsub + 1) * T;
+    const size_t rows = (size_t)B * Hq * (n * nsub) * T;
     best = std::max(best, align_up(rows * D * sizeof(float)) + align_up(rows * sizeof(float)));
   }
   return best;
+}
+
+// Counters of a query chunk's in-kernel reduction and merge: per (head
+// group, query tile) one per context block plus one for the splits; the
+// RoPE launch of the call clears them.
+int chunk_counter_words(int B, int T, int Hq, int Hkv, int Lcap, int block_len) {
+  const int g = Hq / Hkv, hpc = (g % 2 == 0) ? 2 : 1;
+  const long long groups = (long long)B * Hkv * (g / hpc) * ceil_div(T, 128);
+  return (int)(groups * (ceil_div(Lcap, block_len) + 1));
 }
 
 
@@ -196,6 +205,24 @@ namespace star {
 // Sets the calling thread's message for star_last_error (used by entry points
 // defined in other files of the library).
 void set_last_error(const char* msg) { g_err = msg; }
+
+bool encode_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)outer};
+  cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int device_sms() {
+  int sms = 0;
+  return check_device(&sms) == STAR_OK ? sms : 0;
+}
 
 cudaError_t set_smem_attr_once(const void* fn, int slot, int dev, size_t bytes) {
   static std::atomic<bool> done[kAttrSlots][64];
@@ -277,8 +304,9 @@ star_status phase1_run(const void* q, const void* k, const void* v, void* o, voi
                        int block_len, int anchor_len, bool ext, const int32_t* src,
                        const int32_t* pos, int G, const int32_t* bounds, const void* xk,
                        const void* xv, int NX, int ctx_pos0, double theta, void* workspace,
-                       size_t workspace_bytes, void* cuda_stream) {
+                       size_t workspace_bytes, void* cuda_stream, const void* qrot_in = nullptr) {
   star_status s;
+  const bool prerot = qrot_in != nullptr;  // Q rotated and cache rows [0, L) filled by the caller
   if ((s = check_heads(B, Hq, Hkv, D)) != STAR_OK) return s;
   if (L < 1) return fail(STAR_ERR_INVALID_ARG, "L must be >= 1");
   if (block_len < 1) return fail(STAR_ERR_INVALID_ARG, "block_len must be >= 1");
@@ -302,15 +330,22 @@ star_status phase1_run(const void* q, const void* k, const void* v, void* o, voi
                   ctx_pos0);
   }
   if (Lcap < L) return fail(STAR_ERR_INVALID_ARG, "Lcap (%d) < L (%d)", Lcap, L);
-  if (!(theta > 0.0)) return fail(STAR_ERR_INVALID_ARG, "theta must be > 0");
-  if ((s = check_ptr(q, "q")) || (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) ||
-      (s = check_ptr(o, "o")) || (s = check_ptr(k_cache, "k_cache")) ||
-      (s = check_ptr(v_cache, "v_cache")) || (s = check_ptr(workspace, "workspace")))
+  if (!prerot && !(theta > 0.0)) return fail(STAR_ERR_INVALID_ARG, "theta must be > 0");
+  if (prerot) {
+    if ((s = check_ptr(qrot_in, "q_rot")) || (s = check_ptr(o, "o")) ||
+        (s = check_ptr(k_cache, "k_cache")) || (s = check_ptr(v_cache, "v_cache")) ||
+        (s = check_ptr(workspace, "workspace")))
+      return s;
+  } else if ((s = check_ptr(q, "q")) || (s = check_ptr(k, "k")) || (s = check_ptr(v, "v")) ||
+             (s = check_ptr(o, "o")) || (s = check_ptr(k_cache, "k_cache")) ||
+             (s = check_ptr(v_cache, "v_cache")) || (s = check_ptr(workspace, "workspace"))) {
     return s;
+  }
   if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
     return fail(STAR_ERR_INVALID_ARG, "lse is not 4-byte aligned");
-  const size_t need = ext ? star_phase1_ext_workspace_bytes(B, L, Hq, Hkv, D, G)
-                          : star_phase1_workspace_bytes(B, L, Hq, D);
+  const size_t need = prerot ? star::kStatusBytes
+                      : ext  ? star_phase1_ext_workspace_bytes(B, L, Hq, Hkv, D, G)
+                             : star_phase1_workspace_bytes(B, L, Hq, D);
   if (workspace_bytes < need)
     return fail(STAR_ERR_INVALID_ARG, "workspace too small: %zu < %zu bytes", workspace_bytes, need);
   if ((long long)B * Hkv > (1ll << 31) - 1) return fail(STAR_ERR_INVALID_ARG, "B*Hkv too large");
@@ -345,9 +380,11 @@ star_status phase1_run(const void* q, const void* k, const void* v, void* o, voi
   rp.D = D;
   rp.pos = nullptr;
   rp.pos0 = ctx_pos0;  // context row r sits at ctx_pos0 + r
-  star::rope_set_freq(rp, D, theta);
-  e = star::launch_rope(rp, 3, st);
-  if (e != cudaSuccess) return cuda_fail(e, "rope launch");
+  if (!prerot) {
+    star::rope_set_freq(rp, D, theta);
+    e = star::launch_rope(rp, 3, st);
+    if (e != cudaSuccess) return cuda_fail(e, "rope launch");
+  }
   if (ext && G > 0) {
     // the prefix table: K gathered and rotated at pos, V gathered, both
     // head-major [B, Hkv, G, D] in the workspace
@@ -377,7 +414,7 @@ star_status phase1_run(const void* q, const void* k, const void* v, void* o, voi
 
   star::AttnParams ap;
   memset(&ap, 0, sizeof ap);
-  if ((s = map_token_major(&ap.tmQ, qrot, B, L, Hq, D)) != STAR_OK) return s;
+  if ((s = map_token_major(&ap.tmQ, prerot ? qrot_in : qrot, B, L, Hq, D)) != STAR_OK) return s;
   if ((s = map_cache(&ap.tmK, k_cache, B * Hkv, Lcap, L, D, 128)) != STAR_OK) return s;
   if ((s = map_cache(&ap.tmV, v_cache, B * Hkv, Lcap, L, D, 128)) != STAR_OK) return s;
   if (ext && G > 0) {
@@ -439,6 +476,17 @@ star_status star_phase1_encode_ext(const void* q, const void* k, const void* v, 
                     theta, workspace, workspace_bytes, cuda_stream);
 }
 
+star_status star_phase1_encode_rotated(const void* q_rot, void* o, const void* k_cache,
+                                       const void* v_cache, int Lcap, float* lse, int B, int L,
+                                       int Hq, int Hkv, int D, int block_len, int anchor_len,
+                                       void* workspace, size_t workspace_bytes,
+                                       void* cuda_stream) {
+  return phase1_run(nullptr, nullptr, nullptr, o, const_cast<void*>(k_cache),
+                    const_cast<void*>(v_cache), Lcap, lse, B, L, Hq, Hkv, D, block_len, anchor_len,
+                    false, nullptr, nullptr, 0, nullptr, nullptr, nullptr, 0, 0, 1.0, workspace,
+                    workspace_bytes, cuda_stream, q_rot);
+}
+
 size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lcap, int block_len) {
   if (B < 1 || T < 1 || Hq < 1 || Hkv < 1 || D < 1 || Lcap < 1 || block_len < 1 || Hq % Hkv)
     return star::kStatusBytes;
@@ -446,7 +494,8 @@ size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lca
   // in front, so query-chunk and decode calls can share one workspace
   const size_t head = decode_header_bytes(B, Hkv, Lcap, block_len) + align_up((size_t)B * T * Hq * D * 2);
   if (use_decode_path(T, Hq, Hkv)) return head + decode_scratch_bytes(B, Hkv, D, Lcap, block_len);
-  return head + chunk_scratch_bytes(B, T, Hq, Hkv, D, Lcap, block_len);
+  return head + align_up((size_t)chunk_counter_words(B, T, Hq, Hkv, Lcap, block_len) * sizeof(int)) +
+         chunk_scratch_bytes(B, T, Hq, Hkv, D, Lcap, block_len);
 }
 
 }  // extern "C"
@@ -532,7 +581,14 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   rp.pos = nullptr;
   rp.pos0 = q_pos0;
   star::rope_set_freq(rp, D, theta);
+  // query chunks: the counters of the attention kernel's in-kernel reduction
+  // and merge sit after the rotated q; the RoPE launch clears them
+  int* chunk_cnt = reinterpret_cast<int*>(ws + header + qrot_bytes);
+  const int n_cnt = decode ? 0 : chunk_counter_words(B, T, Hq, Hkv, Lcap, block_len);
+  const size_t cnt_bytes = align_up((size_t)n_cnt * sizeof(int));
   if (!decode) {
+    rp.zero = chunk_cnt;
+    rp.nzero = n_cnt;
     e = star::launch_rope(rp, with_tail ? 3 : 1, st);
     if (e != cudaSuccess) return cuda_fail(e, "rope launch");
   }
@@ -609,41 +665,35 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   ap.geom.T = T;
   ap.geom.tail_len = tail_len;
   ap.geom.tail = with_tail;
-  // sub-splits: their partials go to the workspace, then are reduced per split
+  // Blocks cut into sub-splits: the items' partials go to the workspace and
+  // the CTA completing a block reduces them into part_o; the CTA completing
+  // the last split of a (head group, query tile) merges the splits (attend).
+  // One launch after the RoPE kernel.
   const int nsub = chunk_subsplits(B, Hq, Hkv, T, L, block_len, with_tail);
   ap.geom.nsub = nsub;
   ap.geom.sub_len = block_len / nsub;
-  float* sub_o = part_o;
-  float* sub_lse = part_lse;
   if (nsub > 1) {
-    const size_t rows = (size_t)B * Hq * (n * nsub + 1) * T;
-    sub_o = reinterpret_cast<float*>(ws + header + qrot_bytes);
-    sub_lse = reinterpret_cast<float*>(ws + header + qrot_bytes + align_up(rows * D * sizeof(float)));
+    const size_t rows = (size_t)B * Hq * (n * nsub) * T;
+    uint8_t* sub = ws + header + qrot_bytes + cnt_bytes;
+    ap.sub_o = reinterpret_cast<float*>(sub);
+    ap.sub_lse = reinterpret_cast<float*>(sub + align_up(rows * D * sizeof(float)));
   }
+  const int nq = ceil_div(T, 128);
+  ap.cnt_split = chunk_cnt;
+  ap.cnt_group = chunk_cnt + (size_t)ap.geom.groups() * nq * n;
+  ap.o_merged = static_cast<__nv_bfloat16*>(o_merged);
+  ap.lse_merged = o_merged ? lse_merged : nullptr;
   ap.mode = 1;
   ap.num_items = ap.geom.phase2_items();
   ap.qrows = T;
-  ap.nsplit = ap.geom.phase2_splits();
-  ap.part_o = sub_o;
-  ap.part_lse = sub_lse;
+  ap.nsplit = nsplit;
+  ap.part_o = part_o;
+  ap.part_lse = part_lse;
   ap.status = reinterpret_cast<int*>(ws);
   ap.scale_ln = (float)(1.0 / sqrt((double)D));
   ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   e = star::launch_attn(ap, D, st);
   if (e != cudaSuccess) return cuda_fail(e, "phase-2 chunk attention launch");
-  if (nsub > 1) {
-    e = star::launch_subsplit_reduce(sub_o, sub_lse, nsub, n, part_o, part_lse, B, T, Hq, D, st);
-    if (e != cudaSuccess) return cuda_fail(e, "sub-split reduce launch");
-  }
-  if (o_merged) {
-    star::MergeSegs segs{};
-    segs.nseg = 1;
-    segs.slots = nsplit;
-    segs.ns[0] = nsplit;
-    e = star::launch_lse_merge(part_o, part_lse, segs, static_cast<__nv_bfloat16*>(o_merged),
-                               lse_merged, B, T, Hq, D, st);
-    if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
-  }
   return ok();
 }
 

@@ -109,70 +109,6 @@ cudaError_t launch_lse_merge(const float* part_o, const float* part_lse, const M
   return cudaGetLastError();
 }
 
-// Query chunks cut into sub-splits: split s < n combines its sub-split
-// partials s*nsub .. s*nsub + nsub - 1 by the same LSE merge (max first, then
-// weights e^(lse_j - m)) into the split's partial; the tail split n copies
-// sub-split n*nsub. sub_o / sub_lse: [B, Hq, n*nsub + 1, T, D] / [.., T];
-// part_o / part_lse: [B, Hq, n + 1, T, D] / [.., T]. One warp per
-// (batch, head, split, token), lanes over D.
-template <int D>
-__global__ void __launch_bounds__(256) subsplit_reduce_kernel(const float* __restrict__ sub_o,
-                                                              const float* __restrict__ sub_lse,
-                                                              int nsub, int n,
-                                                              float* __restrict__ part_o,
-                                                              float* __restrict__ part_lse, int B,
-                                                              int T, int Hq) {
-  constexpr int kPer = D / 32;
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
-  const int lane = threadIdx.x % 32;
-  const int nsp = n + 1, nss = n * nsub + 1;
-  const long long rows = static_cast<long long>(B) * Hq * nsp * T;
-  if (warp >= rows) return;
-  const int t = warp % T;
-  const int s = (warp / T) % nsp;
-  const size_t bh = static_cast<size_t>(warp) / (static_cast<size_t>(T) * nsp);
-  const int j0 = (s < n) ? s * nsub : n * nsub, cnt = (s < n) ? nsub : 1;
-  auto srow = [&](int j) { return (bh * nss + j) * T + t; };
-  float m = -INFINITY;
-  for (int j = 0; j < cnt; ++j) m = fmaxf(m, sub_lse[srow(j0 + j)]);
-  float acc[kPer];
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) acc[k] = 0.f;
-  float z = 0.f;
-  if (m != -INFINITY) {
-    for (int j = 0; j < cnt; ++j) {
-      const float l = sub_lse[srow(j0 + j)];
-      const float w = (l == -INFINITY) ? 0.f : expf(l - m);
-      z += w;
-      const float* src = sub_o + srow(j0 + j) * D + lane * kPer;
-#pragma unroll
-      for (int k = 0; k < kPer; ++k) acc[k] += w * src[k];
-    }
-  }
-  const float inv = (z > 0.f) ? 1.f / z : 0.f;
-  const size_t prow = (bh * nsp + s) * T + t;
-  float* dst = part_o + prow * D + lane * kPer;
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) dst[k] = acc[k] * inv;
-  if (lane == 0) part_lse[prow] = (z > 0.f) ? m + logf(z) : -INFINITY;
-}
-
-cudaError_t launch_subsplit_reduce(const float* sub_o, const float* sub_lse, int nsub, int n,
-                                   float* part_o, float* part_lse, int B, int T, int Hq, int D,
-                                   cudaStream_t stream) {
-  const long long rows = static_cast<long long>(B) * Hq * (n + 1) * T;
-  if (rows == 0) return cudaSuccess;
-  const int threads = 256;
-  const unsigned blocks = static_cast<unsigned>((rows * 32 + threads - 1) / threads);
-  if (D == 128)
-    subsplit_reduce_kernel<128><<<blocks, threads, 0, stream>>>(sub_o, sub_lse, nsub, n, part_o,
-                                                                part_lse, B, T, Hq);
-  else
-    subsplit_reduce_kernel<64><<<blocks, threads, 0, stream>>>(sub_o, sub_lse, nsub, n, part_o,
-                                                               part_lse, B, T, Hq);
-  return cudaGetLastError();
-}
-
 // Device evaluation of the Phase-1 index math for every context row.
 __global__ void debug_index_kernel(int L, int b, int a, int32_t* blk, int32_t* pos,
                                    int32_t* ranges) {

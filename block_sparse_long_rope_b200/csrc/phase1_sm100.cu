@@ -58,6 +58,155 @@ struct AttnCfg {
 };
 
 constexpr int kAttnThreads = 320;
+
+// ---- Phase-2 query chunks: where an item's rows go, and the in-kernel
+// sub-split reduction and split merge ----------------------------------------
+// An item of a block cut into sub-splits (nsub > 1) writes sub-split row
+// (b, head, split, qrow) of sub_o / sub_lse; any other item (a whole block,
+// or the tail) writes its split's row of part_o / part_lse directly. Returns
+// the row index; *to_sub tells which pair of buffers it indexes.
+__device__ __forceinline__ size_t p2_row(const AttnParams& p, const WorkItem& w, int head, int qrow,
+                                         bool* to_sub) {
+  const AttnGeom& g = p.geom;
+  const size_t bh = static_cast<size_t>(w.b) * g.Hq + head;
+  *to_sub = g.nsub > 1 && w.split < g.n * g.nsub;
+  if (*to_sub) return (bh * (g.n * g.nsub) + w.split) * g.T + qrow;
+  const int api = (w.split < g.n * g.nsub) ? w.split / g.nsub : g.n;
+  return (bh * p.nsplit + api) * g.T + qrow;
+}
+
+// Exact LSE merge of `cnt` partial rows (row(k) indexes lse / o) into one
+// output row: m = max lse_k, w_k = e^(lse_k - m), o = sum w_k o_k / sum w_k,
+// lse = m + log sum w_k, in fixed order [pith 2WVXFXZ2, minor comment on
+// Algorithm 2]. Eight lanes (a quarter warp) take one row, so a warp merges
+// four rows at once; a lane covers D/8 floats as float4s, and the loads of
+// several partials (16 float4s a lane) are issued before they are
+// accumulated. All 32 lanes call it (cnt is the same for the whole warp);
+// `active` is false for a quarter without a row. Writes fp32 (out_o) or bf16
+// (out_b) and the LSE (out_lse, nullable).
+template <int D, typename RowAt>
+__device__ __forceinline__ void merge_rows(int cnt, RowAt row, bool active, const float* lse,
+                                           const float* o, float* out_o, __nv_bfloat16* out_b,
+                                           float* out_lse) {
+  constexpr int kV = D / 32;          // float4s per lane
+  constexpr int kB = 16 / kV;         // partials loaded before use (16 float4s a lane)
+  const int lane = threadIdx.x & 31, q8 = lane & 7, base = lane & 24;
+  float m = -INFINITY;
+  if (active)
+    for (int k = q8; k < cnt; k += 8) m = fmaxf(m, lse[row(k)]);
+#pragma unroll
+  for (int off = 4; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  float4 acc[kV];
+#pragma unroll
+  for (int v = 0; v < kV; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float z = 0.f;
+  for (int k0 = 0; k0 < cnt; k0 += kB) {
+    float wl = 0.f;
+    if (active && q8 < kB && k0 + q8 < cnt && m != -INFINITY) {
+      const float l = lse[row(k0 + q8)];
+      wl = (l == -INFINITY) ? 0.f : expf(l - m);
+    }
+    float zs = wl;
+#pragma unroll
+    for (int off = 4; off > 0; off >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, off);
+    z += zs;
+    float4 x[kB][kV];
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      if (active && k0 + j < cnt) {
+        const float4* src = reinterpret_cast<const float4*>(o + row(k0 + j) * D);
+#pragma unroll
+        for (int v = 0; v < kV; ++v) x[j][v] = src[q8 + 8 * v];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kB; ++j) {
+      const float w = __shfl_sync(0xffffffffu, wl, base + j);
+      if (active && k0 + j < cnt) {
+#pragma unroll
+        for (int v = 0; v < kV; ++v) {
+          acc[v].x += w * x[j][v].x;
+          acc[v].y += w * x[j][v].y;
+          acc[v].z += w * x[j][v].z;
+          acc[v].w += w * x[j][v].w;
+        }
+      }
+    }
+  }
+  if (!active) return;
+  const float inv = (z > 0.f) ? 1.f / z : 0.f;
+#pragma unroll
+  for (int v = 0; v < kV; ++v) {
+    const float4 r = make_float4(acc[v].x * inv, acc[v].y * inv, acc[v].z * inv, acc[v].w * inv);
+    const int c = 4 * (q8 + 8 * v);
+    if (out_o) *reinterpret_cast<float4*>(out_o + c) = r;
+    if (out_b) {
+      uint2 pk;
+      pk.x = pack_bf16x2(r.x, r.y);
+      pk.y = pack_bf16x2(r.z, r.w);
+      *reinterpret_cast<uint2*>(out_b + c) = pk;
+    }
+  }
+  if (out_lse && q8 == 0) *out_lse = (z > 0.f) ? m + logf(z) : -INFINITY;
+}
+
+// Publishes this CTA's writes and counts it in; true for the last of
+// `count` arrivals, after which the others' writes are visible. Every thread
+// of the CTA calls it; one thread touches the counter.
+__device__ __forceinline__ bool count_in_last(int* counter, int count) {
+  __shared__ int s_last;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    s_last = atomicAdd(counter, 1) == count - 1;
+    __threadfence();
+  }
+  __syncthreads();
+  return s_last != 0;
+}
+
+// After a query-chunk item has written its rows: the CTA that completes a
+// block's sub-splits reduces them into the block's split partial; the CTA
+// that completes the last split of a (head group, query tile) merges all
+// splits into o_merged / lse_merged (when asked). All threads of the CTA.
+template <int D>
+__device__ void query_chunk_fold(const AttnParams& p) {
+  const AttnGeom& g = p.geom;
+  const WorkItem w = g.phase2_item(blockIdx.x);  // recomputed: nothing stays live across the loop
+  const int G = g.groups(), nq = g.phase2_qtiles();
+  const int rem = blockIdx.x % (nq * G);
+  const int gq = (rem % G) * nq + rem / G;  // (group, query tile)
+  const int warp = threadIdx.x >> 5, quarter = (threadIdx.x & 31) >> 3;
+  constexpr int kQuarters = kAttnThreads / 8;  // rows merged at once by the CTA
+  const int rows = w.q_hi - w.q_lo, hpc = g.hpc, pairs = rows * hpc;
+  const bool sub = g.nsub > 1 && w.split < g.n * g.nsub;
+  if (sub) {
+    const int blk = w.split / g.nsub;
+    if (!count_in_last(&p.cnt_split[gq * g.n + blk], g.nsub)) return;
+    for (int p0 = 0; p0 < pairs; p0 += kQuarters) {  // warp-uniform trip count
+      const int pr = p0 + 4 * warp + quarter;
+      const bool active = pr < pairs;
+      const int head = w.slot0 + (active ? pr / rows : 0), qrow = w.q_lo + (active ? pr % rows : 0);
+      const size_t bh = static_cast<size_t>(w.b) * g.Hq + head;
+      const size_t s0 = (bh * (g.n * g.nsub) + blk * g.nsub) * g.T + qrow;
+      const size_t out = (bh * p.nsplit + blk) * g.T + qrow;
+      merge_rows<D>(g.nsub, [&](int k) { return s0 + static_cast<size_t>(k) * g.T; }, active,
+                    p.sub_lse, p.sub_o, p.part_o + out * D, nullptr, p.part_lse + out);
+    }
+  }
+  if (p.o_merged == nullptr) return;
+  if (!count_in_last(&p.cnt_group[gq], p.nsplit)) return;
+  for (int p0 = 0; p0 < pairs; p0 += kQuarters) {
+    const int pr = p0 + 4 * warp + quarter;
+    const bool active = pr < pairs;
+    const int head = w.slot0 + (active ? pr / rows : 0), qrow = w.q_lo + (active ? pr % rows : 0);
+    const size_t bh = static_cast<size_t>(w.b) * g.Hq + head;
+    __nv_bfloat16* ob = p.o_merged + ((static_cast<size_t>(w.b) * g.T + qrow) * g.Hq + head) * D;
+    float* lo = p.lse_merged ? p.lse_merged + bh * g.T + qrow : nullptr;
+    merge_rows<D>(p.nsplit, [&](int k) { return (bh * p.nsplit + k) * g.T + qrow; }, active,
+                  p.part_lse, p.part_o, nullptr, ob, lo);
+  }
+}
 constexpr uint64_t kDrainNs = 100000000ull;  // 100 ms
 
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
@@ -69,7 +218,9 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint6
 
 }  // namespace
 
-template <int D>
+// kMode 0: Phase 1; kMode 1: Phase-2 query chunk (one instantiation each,
+// so Phase 1 carries none of the query chunk's epilogue code).
+template <int D, int kMode>
 __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_constant__ AttnParams p) {
   using C = AttnCfg<D>;
   constexpr int S = C::kStages;
@@ -90,7 +241,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
   __shared__ int s_nspan, s_nkv;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const WorkItem w = (p.mode == 0) ? p.geom.phase1_item(blockIdx.x) : p.geom.phase2_item(blockIdx.x);
+  const WorkItem w = (kMode == 0) ? p.geom.phase1_item(blockIdx.x) : p.geom.phase2_item(blockIdx.x);
   const int hpc = p.geom.hpc;
 
   if (threadIdx.x == 0) {
@@ -112,7 +263,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     // the prefix table (clamped to the table; a slice outside it is recorded
     // as a bounds error) and the own block
     int ns = 0;
-    if (p.mode == 0 && p.ext) {
+    if (kMode == 0 && p.ext) {
       const int blk = w.q_lo / p.geom.b;
       if (p.bounds) {
         int gs = p.bounds[2 * blk], ge = p.bounds[2 * blk + 1];
@@ -380,7 +531,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
         tmem_ld32(tO + 32 * q, r);
         tmem_wait_ld();
         reg_fence32(r);
-        if (valid && p.mode == 0) {
+        if (valid && kMode == 0) {
           __nv_bfloat16* dst =
               p.o + ((static_cast<size_t>(b) * p.geom.L + qrow) * Hq + head) * D + 32 * q;
 #pragma unroll
@@ -393,9 +544,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
             reinterpret_cast<uint4*>(dst)[v] = pkd;
           }
         } else if (valid) {
-          const size_t orow =
-              ((static_cast<size_t>(b) * Hq + head) * p.nsplit + w.split) * p.geom.T + qrow;
-          float* dst = p.part_o + orow * D + 32 * q;
+          bool to_sub;
+          const size_t orow = p2_row(p, w, head, qrow, &to_sub);
+          float* dst = (to_sub ? p.sub_o : p.part_o) + orow * D + 32 * q;
 #pragma unroll
           for (int v = 0; v < 8; ++v)
             reinterpret_cast<float4*>(dst)[v] =
@@ -405,10 +556,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
       }
       if (valid) {
         const float lse = (l_run > 0.f) ? m_run * p.scale_ln + logf(l_run) : -INFINITY;
-        if (p.mode == 0) {
+        if (kMode == 0) {
           if (p.lse) p.lse[(static_cast<size_t>(b) * Hq + head) * p.geom.L + qrow] = lse;
         } else {
-          p.part_lse[((static_cast<size_t>(b) * Hq + head) * p.nsplit + w.split) * p.geom.T + qrow] = lse;
+          bool to_sub;
+          const size_t r = p2_row(p, w, head, qrow, &to_sub);
+          (to_sub ? p.sub_lse : p.part_lse)[r] = lse;
         }
       }
     }
@@ -418,6 +571,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   if (warp == 9) tmem_dealloc(tmem, C::kTmemCols);
+  if constexpr (kMode == 1) {
+    if (!abort_flag) query_chunk_fold<D>(p);
+  }
 }
 
 size_t attn_smem_bytes(int D) {
@@ -429,13 +585,19 @@ cudaError_t launch_attn(const AttnParams& p, int D, cudaStream_t stream) {
   const size_t smem = attn_smem_bytes(D);
   int dev = 0;
   cudaGetDevice(&dev);
-  cudaError_t ea = set_smem_attr_once(D == 128 ? (const void*)attn_kernel<128> : (const void*)attn_kernel<64>,
-                                      D == 128 ? 3 : 2, dev, smem);
+  const bool chunk = p.mode == 1;
+  const void* fn = D == 128 ? (chunk ? (const void*)attn_kernel<128, 1> : (const void*)attn_kernel<128, 0>)
+                            : (chunk ? (const void*)attn_kernel<64, 1> : (const void*)attn_kernel<64, 0>);
+  cudaError_t ea = set_smem_attr_once(fn, (D == 128 ? 2 : 0) + (chunk ? 1 : 0), dev, smem);
   if (ea != cudaSuccess) return ea;
-  if (D == 128)
-    attn_kernel<128><<<p.num_items, kAttnThreads, smem, stream>>>(p);
+  if (D == 128 && chunk)
+    attn_kernel<128, 1><<<p.num_items, kAttnThreads, smem, stream>>>(p);
+  else if (D == 128)
+    attn_kernel<128, 0><<<p.num_items, kAttnThreads, smem, stream>>>(p);
+  else if (chunk)
+    attn_kernel<64, 1><<<p.num_items, kAttnThreads, smem, stream>>>(p);
   else
-    attn_kernel<64><<<p.num_items, kAttnThreads, smem, stream>>>(p);
+    attn_kernel<64, 0><<<p.num_items, kAttnThreads, smem, stream>>>(p);
   return cudaGetLastError();
 }
 

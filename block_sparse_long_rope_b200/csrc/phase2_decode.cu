@@ -667,7 +667,7 @@ cudaError_t launch_decode(const DecodeParams& p, int D, cudaStream_t stream) {
   int dev = 0;
   cudaGetDevice(&dev);
   cudaError_t ea = set_smem_attr_once(D == 128 ? (const void*)decode_kernel<128> : (const void*)decode_kernel<64>,
-                                      D == 128 ? 1 : 0, dev, smem);
+                                      D == 128 ? 9 : 8, dev, smem);
   if (ea != cudaSuccess) return ea;
   int sms = 148;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

@@ -21,10 +21,12 @@
 // carries the argument"]).
 //
 // One launch handles up to three jobs (Q, K, V of one call): blockIdx.z
-// selects the job. Each CTA covers kTokPerCta tokens of one job; it first
-// computes the (cos, sin) table of its tokens in shared memory, then streams
-// 16-byte vectors: a thread rotates chunk c of the first half together with
-// chunk c of the second half of one head.
+// selects the job. Each CTA covers p.tpc tokens of one job (8 for long
+// sequences, fewer for a handful of new tokens so that the grid still fills
+// the GPU); it first computes the (cos, sin) table of its tokens in shared
+// memory, then streams 16-byte vectors: a thread rotates chunk c of the first
+// half together with chunk c of the second half of one head. A launch can
+// also clear a few counters of the kernel that follows it (p.zero).
 #include <cmath>
 
 #include "rope_math.cuh"
@@ -35,24 +37,28 @@ namespace star {
 
 namespace {
 constexpr int kRopeThreads = 256;
-constexpr int kTokPerCta = 8;
 }  // namespace
 
 template <int D>
 __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constant__ RopeParams p) {
   constexpr int kHalf = D / 2, kCpr = kHalf / 8;  // 16-byte chunks per half row
   const RopeJob& job = p.job[blockIdx.z];
-  const int tok0 = blockIdx.x * kTokPerCta;
+  if (p.zero) {  // counters of the next kernel in the stream
+    const int cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
+    const int nthr = gridDim.x * gridDim.y * gridDim.z * kRopeThreads;
+    for (int i = cta * kRopeThreads + threadIdx.x; i < p.nzero; i += nthr) p.zero[i] = 0;
+  }
+  const int tok0 = blockIdx.x * p.tpc;
   const int b = blockIdx.y;
-  const int ntok = imin(kTokPerCta, p.S - tok0);
+  const int ntok = imin(p.tpc, p.S - tok0);
   if (ntok <= 0) return;
 
-  __shared__ double s_cos[kTokPerCta][64];
-  __shared__ double s_sin[kTokPerCta][64];
-  __shared__ float f_cos[kTokPerCta][64];
-  __shared__ float f_sin[kTokPerCta][64];
-  __shared__ int s_row[kTokPerCta];  // gather mode: source row, >= 0 in x, < 0 in x2
-  __shared__ int s_ok[kTokPerCta];
+  __shared__ double s_cos[kRopeMaxTok][64];
+  __shared__ double s_sin[kRopeMaxTok][64];
+  __shared__ float f_cos[kRopeMaxTok][64];
+  __shared__ float f_sin[kRopeMaxTok][64];
+  __shared__ int s_row[kRopeMaxTok];  // gather mode: source row, >= 0 in x, < 0 in x2
+  __shared__ int s_ok[kRopeMaxTok];
   if (p.src) {
     if (threadIdx.x < ntok) {
       const int r = p.src[tok0 + threadIdx.x];
@@ -132,9 +138,16 @@ void rope_fill_freq(double* out, int D, double theta) {
     out[i] = (i < D / 2) ? std::pow(theta, -2.0 * static_cast<double>(i) / static_cast<double>(D)) : 0.0;
 }
 
-cudaError_t launch_rope(const RopeParams& p, int njobs, cudaStream_t stream) {
-  if (njobs <= 0 || p.S <= 0 || p.B <= 0) return cudaSuccess;
-  dim3 grid(ceil_div(p.S, kTokPerCta), p.B, njobs);
+cudaError_t launch_rope(const RopeParams& p_in, int njobs, cudaStream_t stream) {
+  if (njobs <= 0 || p_in.S <= 0 || p_in.B <= 0) return cudaSuccess;
+  RopeParams p = p_in;
+  if (p.tpc <= 0 || p.tpc > kRopeMaxTok) {
+    // 8 tokens per CTA amortise the cos/sin table; a short call (a query
+    // chunk) takes fewer so that its grid still covers two waves of CTAs
+    p.tpc = kRopeMaxTok;
+    while (p.tpc > 1 && (long long)ceil_div(p.S, p.tpc) * p.B * njobs < 2 * 148) p.tpc /= 2;
+  }
+  dim3 grid(ceil_div(p.S, p.tpc), p.B, njobs);
   if (p.D == 128)
     rope_kernel<128><<<grid, kRopeThreads, 0, stream>>>(p);
   else

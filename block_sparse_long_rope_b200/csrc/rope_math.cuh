@@ -56,11 +56,11 @@ __device__ __forceinline__ uint32_t rope_rotate_bf16(float a, float b, float c32
 
 // Both outputs of one pair: low 16 bits the bf16 of a*c - b*s, high 16 bits
 // that of b*c + a*s, each correctly rounded exactly as rope_rotate_bf16 does.
-// The error bound is shared, and the fp64 cos/sin (c64, s64: read through
-// the pointers) are loaded only when a result is within the bound of a
-// rounding boundary.
-__device__ __forceinline__ uint32_t rope_rotate_pair_bf16(float a, float b, float c32, float s32,
-                                                          const double* c64, const double* s64) {
+// The error bound is shared, and the fp64 cos/sin are fetched (get64(&c,
+// &s)) only when a result is within the bound of a rounding boundary.
+template <typename Get64>
+__device__ __forceinline__ uint32_t rope_rotate_pair_bf16_with(float a, float b, float c32,
+                                                               float s32, Get64 get64) {
   const float e = 2.3841858e-07f * (fabsf(a) + fabsf(b));
   const float y0 = fmaf(a, c32, -(b * s32));
   const float y1 = fmaf(b, c32, a * s32);
@@ -68,11 +68,30 @@ __device__ __forceinline__ uint32_t rope_rotate_pair_bf16(float a, float b, floa
   uint32_t o0 = r0 & 0xFFFFu, o1 = r1 & 0xFFFFu;
   const bool ok0 = o0 == (r0 >> 16), ok1 = o1 == (r1 >> 16);
   if (!(ok0 && ok1)) {
-    const double ad = a, bd = b, cd = *c64, sd = *s64;
+    double cd, sd;
+    get64(&cd, &sd);
+    const double ad = a, bd = b;
     if (!ok0) o0 = pack_bf16x2(f32_round_odd(ad * cd - bd * sd), 0.f) & 0xFFFFu;
     if (!ok1) o1 = pack_bf16x2(f32_round_odd(bd * cd + ad * sd), 0.f) & 0xFFFFu;
   }
   return o0 | (o1 << 16);
+}
+
+// As above with the fp64 cos/sin read through pointers (from a table).
+__device__ __forceinline__ uint32_t rope_rotate_pair_bf16(float a, float b, float c32, float s32,
+                                                          const double* c64, const double* s64) {
+  return rope_rotate_pair_bf16_with(a, b, c32, s32, [&](double* c, double* s) {
+    *c = *c64;
+    *s = *s64;
+  });
+}
+
+// As above with the fp64 cos/sin of pos * inv_freq recomputed on the rare
+// slow path (c32/s32 must be the fp32 roundings of rope_angle's results).
+__device__ __forceinline__ uint32_t rope_rotate_pair_bf16_at(float a, float b, float c32, float s32,
+                                                             long long pos, double inv_freq) {
+  return rope_rotate_pair_bf16_with(a, b, c32, s32,
+                                    [&](double* c, double* s) { rope_angle(pos, inv_freq, c, s); });
 }
 
 }  // namespace star

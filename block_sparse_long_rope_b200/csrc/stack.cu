@@ -8,16 +8,16 @@
 //
 // RMSNorm: one CTA per row, fp32 sum of squares, y = x * rsqrt(mean(x^2) +
 // eps) * gamma rounded to bf16. HBM-bound.
-// Projections: plain GEMMs, y[M, N] (+)= x[M, K] * w[N, K]^T in bf16 with fp32
-// accumulation, through cuBLASLt; the residual is its beta = 1 term. Split-K
-// algorithms are limited to fp32 reductions, so the only bf16 rounding is the
-// final one.
-#include <cublasLt.h>
-
+// Projections: the library's tcgen05 GEMM (gemm_sm100.cu), y[M, N] (+)=
+// x[M, K] * w[N, K]^T in bf16 with fp32 accumulation; the residual add rounds
+// the bf16 projection plus y once more. star_linear_rope adds the RoPE and
+// KV-cache epilogues, so a layer's Q and K leave the projection already
+// rotated and K/V land in the cache without a separate pass.
+#include <cmath>
 #include <cstdio>
-#include <map>
-#include <mutex>
-#include <tuple>
+
+#include <cstdarg>
+#include <cstring>
 
 #include "star.h"
 #include "star_common.cuh"
@@ -70,23 +70,6 @@ __global__ void __launch_bounds__(kNormThreads) rmsnorm_kernel(const __nv_bfloat
   }
 }
 
-// ---- cuBLASLt --------------------------------------------------------------
-std::mutex g_lt_mu;
-cublasLtHandle_t g_lt = nullptr;
-using AlgoKey = std::tuple<int, int, int, int, int, size_t>;  // device, M, N, K, beta, workspace
-std::map<AlgoKey, cublasLtMatmulAlgo_t> g_algos;
-
-struct LtDescs {
-  cublasLtMatmulDesc_t op = nullptr;
-  cublasLtMatrixLayout_t a = nullptr, b = nullptr, c = nullptr;
-  ~LtDescs() {
-    if (c) cublasLtMatrixLayoutDestroy(c);
-    if (b) cublasLtMatrixLayoutDestroy(b);
-    if (a) cublasLtMatrixLayoutDestroy(a);
-    if (op) cublasLtMatmulDescDestroy(op);
-  }
-};
-
 }  // namespace
 
 cudaError_t launch_rmsnorm(const __nv_bfloat16* x, const __nv_bfloat16* gamma, __nv_bfloat16* y,
@@ -99,12 +82,70 @@ cudaError_t launch_rmsnorm(const __nv_bfloat16* x, const __nv_bfloat16* gamma, _
 }  // namespace star
 
 namespace {
-star_status lt_fail(cublasStatus_t st, const char* what) {
-  char buf[256];
-  snprintf(buf, sizeof buf, "cuBLASLt %s failed (status %d)", what, static_cast<int>(st));
+
+star_status stack_fail(star_status st, const char* fmt, ...) {
+  char buf[320];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
   star::set_last_error(buf);
-  return STAR_ERR_CUDA;
+  return st;
 }
+
+bool misaligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0; }
+
+// Shared body of star_linear / star_linear_rope: checks, TMA maps, launch.
+star_status run_gemm(const void* x, const void* w, void* y, int M, int N, int K, int accumulate,
+                     int head_dim, int rotate, int seq_len, long long pos0, double theta,
+                     int cache_rows, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  if (M < 1 || N < 1 || K < 1 || N % 8 || K % 8)
+    return stack_fail(STAR_ERR_INVALID_ARG, "bad shape M=%d N=%d K=%d (N, K multiples of 8)", M, N, K);
+  if (!x || !w || !y || misaligned(x, 16) || misaligned(w, 16) || misaligned(y, 16))
+    return stack_fail(STAR_ERR_INVALID_ARG, "x, w and y must be non-NULL and 16-byte aligned");
+  const size_t need = star_linear_rope_workspace_bytes(seq_len, head_dim, rotate);
+  if (!workspace || workspace_bytes < need || misaligned(workspace, 256))
+    return stack_fail(STAR_ERR_INVALID_ARG,
+                      "workspace must be 256-byte aligned with >= %zu bytes (status word%s)", need,
+                      rotate ? " and cos/sin table" : "");
+  if ((long long)M * N > (1ll << 46) || (long long)M * K > (1ll << 46) || (long long)N * K > (1ll << 46))
+    return stack_fail(STAR_ERR_INVALID_ARG, "problem too large");
+  const int sms = star::device_sms();
+  if (sms <= 0) return STAR_ERR_UNSUPPORTED;  // message set by the device check
+  star::GemmParams p;
+  memset(&p, 0, sizeof p);
+  if (!star::encode_tmap_2d(&p.tmA, x, (uint64_t)K, (uint64_t)M, (uint64_t)K * 2, 64, 128) ||
+      !star::encode_tmap_2d(&p.tmB, w, (uint64_t)K, (uint64_t)N, (uint64_t)K * 2, 64, 256))
+    return stack_fail(STAR_ERR_CUDA, "cuTensorMapEncodeTiled failed for the GEMM operands");
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.m_tiles = (M + 127) / 128;
+  p.n_tiles = (N + 255) / 256;
+  p.k_blocks = (K + 63) / 64;
+  p.y = static_cast<__nv_bfloat16*>(y);
+  p.accumulate = accumulate;
+  p.rd = rotate ? head_dim : 0;
+  p.hd = head_dim;
+  p.seq_len = seq_len;
+  p.cache_rows = cache_rows;
+  p.pos0 = pos0;
+  p.status = static_cast<int*>(workspace);
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  cudaError_t e;
+  if (rotate) {
+    star::rope_fill_freq(p.inv_freq, head_dim, theta);
+    float2* tab = reinterpret_cast<float2*>(static_cast<uint8_t*>(workspace) + star::kStatusBytes);
+    e = star::launch_rope_table(tab, seq_len, head_dim / 2, pos0, p.inv_freq, st);
+    if (e != cudaSuccess) return stack_fail(STAR_ERR_CUDA, "rope table launch: %s", cudaGetErrorString(e));
+    p.rope_tab = tab;
+  }
+  e = star::launch_gemm(p, sms, st);
+  if (e != cudaSuccess) return stack_fail(STAR_ERR_CUDA, "gemm launch: %s", cudaGetErrorString(e));
+  star::set_last_error("");
+  return STAR_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -135,84 +176,40 @@ star_status star_rmsnorm(const void* x, const void* gamma, void* y, int rows, in
   return STAR_OK;
 }
 
+size_t star_linear_rope_workspace_bytes(int seq_len, int head_dim, int rotate) {
+  if (!rotate || seq_len < 1 || head_dim < 2) return star::kStatusBytes;
+  const size_t tab = (size_t)seq_len * (head_dim / 2) * 8;
+  return star::kStatusBytes + (tab + 255) / 256 * 256;
+}
+
 star_status star_linear(const void* x, const void* w, void* y, int M, int N, int K, int accumulate,
                         void* workspace, size_t workspace_bytes, void* cuda_stream) {
-  char buf[256];
-  if (M < 1 || N < 1 || K < 1 || N % 8 || K % 8 || (accumulate != 0 && accumulate != 1)) {
-    snprintf(buf, sizeof buf, "bad shape M=%d N=%d K=%d (N, K multiples of 8) accumulate=%d", M,
-             N, K, accumulate);
-    star::set_last_error(buf);
-    return STAR_ERR_INVALID_ARG;
-  }
-  if (!x || !w || !y || (reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(w) |
-                         reinterpret_cast<uintptr_t>(y)) & 15u) {
-    star::set_last_error("x, w and y must be non-NULL and 16-byte aligned");
-    return STAR_ERR_INVALID_ARG;
-  }
-  if (workspace_bytes && (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))) {
-    star::set_last_error("workspace must be 256-byte aligned when workspace_bytes > 0");
-    return STAR_ERR_INVALID_ARG;
-  }
-  int dev = 0;
-  cudaError_t ce = cudaGetDevice(&dev);
-  if (ce != cudaSuccess) {
-    snprintf(buf, sizeof buf, "no CUDA device: %s", cudaGetErrorString(ce));
-    star::set_last_error(buf);
-    return STAR_ERR_CUDA;
-  }
-  cublasStatus_t st;
-  {
-    std::lock_guard<std::mutex> lk(star::g_lt_mu);
-    if (!star::g_lt && (st = cublasLtCreate(&star::g_lt)) != CUBLAS_STATUS_SUCCESS)
-      return lt_fail(st, "create");
-  }
-  // row-major y[M, N] = x[M, K] w[N, K]^T, read column-major, is
-  // y^T (N x M) = A^T B with A = w stored K x N (ld K) and B = x stored
-  // K x M (ld K); C = D = y stored N x M (ld N)
-  star::LtDescs d;
-  const cublasOperation_t ta = CUBLAS_OP_T, tb = CUBLAS_OP_N;
-  if ((st = cublasLtMatmulDescCreate(&d.op, CUBLAS_COMPUTE_32F, CUDA_R_32F)) ||
-      (st = cublasLtMatmulDescSetAttribute(d.op, CUBLASLT_MATMUL_DESC_TRANSA, &ta, sizeof ta)) ||
-      (st = cublasLtMatmulDescSetAttribute(d.op, CUBLASLT_MATMUL_DESC_TRANSB, &tb, sizeof tb)) ||
-      (st = cublasLtMatrixLayoutCreate(&d.a, CUDA_R_16BF, K, N, K)) ||
-      (st = cublasLtMatrixLayoutCreate(&d.b, CUDA_R_16BF, K, M, K)) ||
-      (st = cublasLtMatrixLayoutCreate(&d.c, CUDA_R_16BF, N, M, N)))
-    return lt_fail(st, "descriptor");
-  const star::AlgoKey key{dev, M, N, K, accumulate, workspace_bytes};
-  cublasLtMatmulAlgo_t algo;
-  {
-    std::lock_guard<std::mutex> lk(star::g_lt_mu);
-    auto it = star::g_algos.find(key);
-    if (it == star::g_algos.end()) {
-      cublasLtMatmulPreference_t pref = nullptr;
-      cublasLtMatmulHeuristicResult_t res{};
-      int nres = 0;
-      st = cublasLtMatmulPreferenceCreate(&pref);
-      if (st == CUBLAS_STATUS_SUCCESS)
-        st = cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_MAX_WORKSPACE_BYTES,
-                                                  &workspace_bytes, sizeof workspace_bytes);
-      // split-K partial sums stay in fp32: no in-place reduction in the bf16
-      // output (which would round every partial sum)
-      const uint32_t schemes = CUBLASLT_REDUCTION_SCHEME_NONE | CUBLASLT_REDUCTION_SCHEME_COMPUTE_TYPE;
-      if (st == CUBLAS_STATUS_SUCCESS)
-        st = cublasLtMatmulPreferenceSetAttribute(pref, CUBLASLT_MATMUL_PREF_REDUCTION_SCHEME_MASK,
-                                                  &schemes, sizeof schemes);
-      if (st == CUBLAS_STATUS_SUCCESS)
-        st = cublasLtMatmulAlgoGetHeuristic(star::g_lt, d.op, d.a, d.b, d.c, d.c, pref, 1, &res,
-                                            &nres);
-      if (pref) cublasLtMatmulPreferenceDestroy(pref);
-      if (st != CUBLAS_STATUS_SUCCESS) return lt_fail(st, "heuristic");
-      if (nres < 1) return lt_fail(CUBLAS_STATUS_NOT_SUPPORTED, "heuristic (no algorithm)");
-      it = star::g_algos.emplace(key, res.algo).first;
-    }
-    algo = it->second;
-  }
-  const float alpha = 1.f, beta = accumulate ? 1.f : 0.f;
-  st = cublasLtMatmul(star::g_lt, d.op, &alpha, w, d.a, x, d.b, &beta, y, d.c, y, d.c, &algo,
-                      workspace, workspace_bytes, static_cast<cudaStream_t>(cuda_stream));
-  if (st != CUBLAS_STATUS_SUCCESS) return lt_fail(st, "matmul");
-  star::set_last_error("");
-  return STAR_OK;
+  if (accumulate != 0 && accumulate != 1)
+    return stack_fail(STAR_ERR_INVALID_ARG, "accumulate must be 0 or 1 (got %d)", accumulate);
+  return run_gemm(x, w, y, M, N, K, accumulate, 64, 0, M, 0, 1.0, 0, workspace, workspace_bytes,
+                  cuda_stream);
+}
+
+star_status star_linear_rope(const void* x, const void* w, void* y, int M, int N, int K,
+                             int head_dim, int rotate, int seq_len, int64_t pos0, double theta,
+                             int cache_rows, void* workspace, size_t workspace_bytes,
+                             void* cuda_stream) {
+  if (head_dim != 64 && head_dim != 128)
+    return stack_fail(STAR_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", head_dim);
+  if (rotate != 0 && rotate != 1)
+    return stack_fail(STAR_ERR_INVALID_ARG, "rotate must be 0 or 1 (got %d)", rotate);
+  if (N % head_dim) return stack_fail(STAR_ERR_INVALID_ARG, "N (%d) must be whole heads of %d", N, head_dim);
+  if (seq_len < 1 || M % seq_len)
+    return stack_fail(STAR_ERR_INVALID_ARG, "M (%d) must be a multiple of seq_len (%d)", M, seq_len);
+  if (cache_rows != 0 && cache_rows < seq_len)
+    return stack_fail(STAR_ERR_INVALID_ARG, "cache_rows (%d) must be 0 or >= seq_len (%d)",
+                      cache_rows, seq_len);
+  if (!rotate && cache_rows == 0)
+    return stack_fail(STAR_ERR_INVALID_ARG, "neither rotation nor a cache layout: use star_linear");
+  if (rotate && (pos0 < 0 || !(theta > 0.0)))
+    return stack_fail(STAR_ERR_INVALID_ARG, "pos0 must be >= 0 and theta > 0");
+  return run_gemm(x, w, y, M, N, K, 0, head_dim, rotate, seq_len, pos0, theta, cache_rows,
+                  workspace, workspace_bytes, cuda_stream);
 }
 
 }  // extern "C"

@@ -26,6 +26,7 @@ struct RopeJob {
 struct RopeParams {
   RopeJob job[3];
   int B, S, D;
+  int tpc;             // tokens per CTA (1..kRopeMaxTok; launch_rope picks it when 0)
   const int32_t* pos;  // nullable: position of token s is pos0 + s
   long long pos0;
   // gather mode (src != nullptr): output token s reads row src[s] of x when
@@ -34,8 +35,11 @@ struct RopeParams {
   const int32_t* src;
   int nsrc, nx;
   int* status;
+  int* zero;   // nullable: nzero ints cleared by the launch (counters of the next kernel)
+  int nzero;
   double inv_freq[64];  // theta^(-2i/D), i < D/2 (fp64, from the host)
 };
+constexpr int kRopeMaxTok = 8;
 // Fills out[0..63] with theta^(-2i/D) for i < D/2 (zero beyond).
 void rope_fill_freq(double* out, int D, double theta);
 inline void rope_set_freq(RopeParams& p, int D, double theta) { rope_fill_freq(p.inv_freq, D, theta); }
@@ -58,8 +62,17 @@ struct AttnParams {
   int nsplit;
   __nv_bfloat16* o;  // Phase 1: [B, L, Hq, D]
   float* lse;        // Phase 1: [B, Hq, L] (nullable)
-  float* part_o;     // Phase 2: [B, Hq, nsplit, T, D]
+  float* part_o;     // Phase 2: [B, Hq, nsplit, T, D], nsplit = n + tail (the API's splits)
   float* part_lse;   // Phase 2: [B, Hq, nsplit, T]
+  // Phase-2 query chunks whose blocks are cut into nsub sub-splits: the
+  // items' partials go to sub_o / sub_lse ([B, Hq, n * nsub, T, D] / [.., T]);
+  // the CTA finishing a block's last sub-split reduces them into part_o.
+  float* sub_o;
+  float* sub_lse;
+  int* cnt_split;    // [groups, qtiles, n] finished sub-splits (cleared by the RoPE launch)
+  int* cnt_group;    // [groups, qtiles] finished splits (cleared by the RoPE launch)
+  __nv_bfloat16* o_merged;  // nullable: [B, T, Hq, D]; the CTA finishing the last split merges
+  float* lse_merged;        // nullable: [B, Hq, T]
   int* status;
   float scale_log2;  // log2(e) / sqrt(D)
   float scale_ln;    // 1 / sqrt(D)
@@ -116,9 +129,30 @@ struct MergeSegs {
 cudaError_t launch_lse_merge(const float* part_o, const float* part_lse, const MergeSegs& segs,
                              __nv_bfloat16* o, float* lse, int B, int T, int Hq, int D,
                              cudaStream_t stream);
-cudaError_t launch_subsplit_reduce(const float* sub_o, const float* sub_lse, int nsub, int n,
-                                   float* part_o, float* part_lse, int B, int T, int Hq, int D,
-                                   cudaStream_t stream);
+
+// ---- projection GEMM (tcgen05): y[M, N] = x[M, K] w[N, K]^T with epilogues --
+struct GemmParams {
+  CUtensorMap tmA;  // x [M, K] row-major: dims {K, M}, box {64, 128}
+  CUtensorMap tmB;  // w [N, K] row-major: dims {K, N}, box {64, 256}
+  int M, N, K;
+  int m_tiles, n_tiles, k_blocks;  // 128-row, 256-column and 64-deep tiles
+  __nv_bfloat16* y;
+  int accumulate;   // 1: y = bf16(y + bf16(acc)) (row-major, no rotation)
+  int rd;           // 64 / 128: rotate every rd-column head (RoPE); 0: no rotation
+  int hd;           // head dim of the cache layout (cache_rows > 0)
+  int seq_len;      // rows per sequence: row m is token m % seq_len of sequence m / seq_len
+  int cache_rows;   // 0: y row-major [M, N]; > 0: y head-major [M / seq_len, N / hd, cache_rows, hd]
+  long long pos0;   // RoPE position of token t = pos0 + t
+  double inv_freq[64];  // theta^(-2i/rd), i < rd/2
+  const float2* rope_tab;  // [seq_len][rd/2] fp32 roundings of (cos, sin)(pos * inv_freq)
+  int* status;      // device status word (bounded waits)
+};
+size_t gemm_smem_bytes();
+cudaError_t launch_gemm(const GemmParams& p, int sms, cudaStream_t stream);
+// Fills tab[t][i] = fp32 roundings of the fp64 (cos, sin) of (pos0 + t) *
+// inv_freq[i] (rope_angle), t < S, i < half.
+cudaError_t launch_rope_table(float2* tab, int S, int half, long long pos0, const double* inv_freq,
+                              cudaStream_t stream);
 
 // ---- error message of the calling thread (star_last_error) -------------------
 void set_last_error(const char* msg);
@@ -128,8 +162,16 @@ void set_last_error(const char* msg);
 // the first time it is asked for that (slot, device); later calls return at
 // once. Safe to call from several host threads. slot < kAttrSlots names the
 // kernel (one slot per kernel instantiation).
-constexpr int kAttrSlots = 8;
+constexpr int kAttrSlots = 16;  // attention 0-3, GEMM 4-6, decode 8-9
 cudaError_t set_smem_attr_once(const void* fn, int slot, int dev, size_t bytes);
+// Rank-2 TMA map of a row-major bf16 matrix (inner x outer elements, rows
+// row_bytes apart) with a box of box_inner x box_outer and 128-byte swizzle;
+// false if the driver rejects it.
+bool encode_tmap_2d(CUtensorMap* m, const void* base, uint64_t inner, uint64_t outer,
+                    uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
+// SM count of the current device if it is supported (sm_100), else 0 (the
+// message is then set for star_last_error).
+int device_sms();
 
 // ---- debug: device-evaluated index math --------------------------------------
 cudaError_t launch_debug_index(int L, int b, int a, int32_t* blk, int32_t* pos, int32_t* ranges,

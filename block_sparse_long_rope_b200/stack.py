@@ -20,7 +20,6 @@ from . import star
 from .configs import Workload
 from .pipeline import StarLayer
 
-GEMM_WORKSPACE = 32 << 20
 
 
 class StarStack:
@@ -36,25 +35,33 @@ class StarStack:
         bf = dict(dtype=torch.bfloat16, device=dev)
         self.h = torch.empty((B, L, dm), **bf)
         self.q = torch.empty((B, L, Hq, D), **bf)
-        self.k = torch.empty((B, L, Hkv, D), **bf)
-        self.v = torch.empty((B, L, Hkv, D), **bf)
         Tmax = max(w.Tq, 1)
         self.h2 = torch.empty((B * Tmax * dm,), **bf)
         self.q2 = torch.empty((B * Tmax * Hq * D,), **bf)
         self.k2 = torch.empty((B * Tmax * Hkv * D,), **bf)
         self.v2 = torch.empty((B * Tmax * Hkv * D,), **bf)
-        self.gemm_ws = star.alloc_workspace(GEMM_WORKSPACE, dev)
+        # the GEMMs' status word and the RoPE epilogue's cos/sin table
+        self.gemm_ws = star.alloc_workspace(
+            star.star_linear_rope_workspace_bytes(max(L, Tmax), D, True), dev)
 
     def encode_layer(self, x, index):
         """Phase 1 of layer `index` on the residual stream x [B, L, dm] bf16
-        (updated in place); fills that layer's KV cache rows [0, L)."""
+        (updated in place); fills that layer's KV cache rows [0, L). The Q
+        projection leaves Q rotated, the K and V projections write the
+        layer's cache (K rotated) directly, then only the attention runs."""
+        w = self.w
         ly, wt = self.layers[index], self.weights[index]
+        b = ly.buf
         star.star_rmsnorm(x, wt["gamma"], self.h, self.eps)
-        star.star_linear(self.h, wt["wq"], self.q, workspace=self.gemm_ws)
-        star.star_linear(self.h, wt["wk"], self.k, workspace=self.gemm_ws)
-        star.star_linear(self.h, wt["wv"], self.v, workspace=self.gemm_ws)
-        o = ly.encode(self.q, self.k, self.v, with_lse=False)
-        star.star_linear(o, wt["wo"], x, accumulate=True, workspace=self.gemm_ws)
+        star.star_linear_rope(self.h, wt["wq"], self.q, w.D, True, w.L, 0, w.theta, 0,
+                              self.gemm_ws)
+        star.star_linear_rope(self.h, wt["wk"], b.k_cache, w.D, True, w.L, 0, w.theta, w.Lcap,
+                              self.gemm_ws)
+        star.star_linear_rope(self.h, wt["wv"], b.v_cache, w.D, False, w.L, 0, w.theta, w.Lcap,
+                              self.gemm_ws)
+        star.star_phase1_encode_rotated(self.q, b.o, b.k_cache, b.v_cache, w.L, w.block_len,
+                                        w.anchor_len, b.ws1)
+        star.star_linear(b.o, wt["wo"], x, accumulate=True, workspace=self.gemm_ws)
         return x
 
     def encode(self, x):

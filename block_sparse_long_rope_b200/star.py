@@ -277,6 +277,49 @@ def star_linear(x, w, y, accumulate=False, workspace=None, stream=None):
     return y
 
 
+def star_linear_rope(x, w, y, head_dim, rotate, seq_len, pos0, theta, cache_rows, workspace,
+                     stream=None):
+    """A projection p = bf16(x[M, K] w[N, K]^T) whose heads of head_dim
+    columns are RoPE'd (rotate) at positions pos0 + row % seq_len and/or
+    stored head-major into a KV cache [M / seq_len, N / head_dim,
+    cache_rows, head_dim] (cache_rows > 0); y row-major [M, N] otherwise."""
+    for t, n in ((x, "x"), (w, "w"), (y, "y")):
+        _bf16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    N, K = w.shape
+    M = x.numel() // K
+    lib = _abi.load()
+    _abi.check(lib.star_linear_rope(_ptr(x), _ptr(w), _ptr(y), M, N, K, int(head_dim),
+                                    1 if rotate else 0, int(seq_len), int(pos0), float(theta),
+                                    int(cache_rows), _ptr(workspace),
+                                    workspace.numel() * workspace.element_size(), _stream(stream)))
+    return y
+
+
+def star_linear_rope_workspace_bytes(seq_len, head_dim, rotate) -> int:
+    return int(_abi.load().star_linear_rope_workspace_bytes(int(seq_len), int(head_dim),
+                                                            1 if rotate else 0))
+
+
+def star_phase1_encode_rotated(q_rot, o, k_cache, v_cache, L, block_len, anchor_len, workspace,
+                               lse=None, stream=None):
+    """Phase 1 attention when q_rot[B,L,Hq,D] is already rotated and cache rows
+    [0, L) hold the rotated keys and the values (see star_linear_rope)."""
+    for t, n in ((q_rot, "q_rot"), (o, "o"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _bf16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    B, Lq, Hq, D = q_rot.shape
+    Hkv, Lcap = k_cache.shape[1], k_cache.shape[2]
+    lib = _abi.load()
+    _abi.check(lib.star_phase1_encode_rotated(
+        _ptr(q_rot), _ptr(o), _ptr(k_cache), _ptr(v_cache), Lcap, _ptr(lse), B, int(L), Hq, Hkv,
+        D, int(block_len), int(anchor_len), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return o
+
+
 def star_device_status(workspace, stream=None):
     """Synchronise, read and clear the device status word; raises on a device error."""
     lib = _abi.load()

@@ -132,6 +132,21 @@ star_status star_phase1_encode(const void* q, const void* k, const void* v, void
                                double theta, void* workspace, size_t workspace_bytes,
                                void* cuda_stream);
 
+/*
+ * star_phase1_encode_rotated — star_phase1_encode when the caller has already
+ * rotated Q and written the cache (for example with star_linear_rope):
+ * q_rot[B, L, Hq, D] holds RoPE'd queries at positions 0..L-1 and
+ * k_cache/v_cache[B, Hkv, Lcap, D] rows [0, L) hold the rotated keys and the
+ * values. Only the block-sparse attention runs; the visibility rule, o and
+ * lse are those of star_phase1_encode. workspace: >= 256 bytes (the status
+ * word), zero-filled once. Errors as star_phase1_encode.
+ */
+star_status star_phase1_encode_rotated(const void* q_rot, void* o, const void* k_cache,
+                                       const void* v_cache, int Lcap, float* lse, int B, int L,
+                                       int Hq, int Hkv, int D, int block_len, int anchor_len,
+                                       void* workspace, size_t workspace_bytes,
+                                       void* cuda_stream);
+
 /* Workspace bytes star_phase1_encode_ext needs for a prefix table of G
  * rows: as star_phase1_encode plus the table's rotated K and its V (bf16
  * [B, Hkv, G, D] each). */
@@ -342,19 +357,50 @@ star_status star_phase2_decode_static_status(void* cuda_stream);
  *   arithmetic, one rounding to bf16. dm a multiple of 8, pointers 16-byte
  *   aligned. STAR_ERR_INVALID_ARG otherwise; STAR_ERR_CUDA if the launch fails.
  *
- * star_linear — y[M, N] = x[M, K] * w[N, K]^T (+ y[M, N] if accumulate = 1,
- *   the residual add), bf16 row-major operands, fp32 accumulation, one
- *   rounding to bf16. A plain GEMM: it runs in cuBLASLt. N and K multiples of
- *   8, pointers 16-byte aligned; workspace (optional, caller-owned, 256-byte
- *   aligned) is cuBLASLt's scratch. The library keeps one cuBLASLt handle and
- *   a cache of chosen algorithms per (device, shape); it allocates no device
- *   memory. STAR_ERR_INVALID_ARG for bad shapes or pointers, STAR_ERR_CUDA for
- *   a cuBLASLt failure (message names the step).
+ * star_linear — y[M, N] = x[M, K] * w[N, K]^T (accumulate = 0), or
+ *   y = bf16(y + bf16(x * w^T)) (accumulate = 1: the stored projection, then
+ *   the residual add), bf16 row-major operands, fp32 accumulation. It runs in
+ *   the library's own tcgen05 GEMM (128 x 256 tiles, TMA-fed, persistent).
+ *   N and K multiples of 8, x/w/y 16-byte aligned. workspace (caller-owned,
+ *   256-byte aligned, >= 256 bytes, zero-filled once) holds the status word a
+ *   bounded wait writes on a time-out (star_device_status reads it).
+ *   STAR_ERR_INVALID_ARG for bad shapes or pointers, STAR_ERR_UNSUPPORTED off
+ *   sm_100, STAR_ERR_CUDA for a failed launch.
  */
 star_status star_rmsnorm(const void* x, const void* gamma, void* y, int rows, int dm, float eps,
                          void* cuda_stream);
 star_status star_linear(const void* x, const void* w, void* y, int M, int N, int K, int accumulate,
                         void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/*
+ * star_linear_rope — a Q/K/V projection whose output goes straight to where
+ * Star attention reads it [pith 2WVXFXZ2, "What carries the argument": keys
+ * keep their original position IDs; pith 2607.20457: original global
+ * positions preserve RoPE distances]:
+ *   p = bf16(x[M, K] * w[N, K]^T), rows m = b * seq_len + t (token t of
+ *   sequence b), N = H * head_dim columns (H heads);
+ *   rotate = 1: every head is rotated as star_rope does (rotate-half, base
+ *   theta, position pos0 + t), from the bf16 values p, correctly rounded, so
+ *   the bits equal star_linear followed by star_rope;
+ *   cache_rows = 0: y is row-major [M, N] (token-major [B, seq_len, H, D]);
+ *   cache_rows > 0: y is a head-major KV cache [B, H, cache_rows, head_dim]
+ *   and token t of sequence b lands in row t (rows >= seq_len untouched).
+ * A Phase-1 layer projects Q with rotate = 1, cache_rows = 0, K with
+ * rotate = 1 into its k_cache and V with rotate = 0 into its v_cache, then
+ * calls star_phase1_encode_rotated: no separate RoPE pass.
+ * head_dim 64 or 128; N a multiple of head_dim; M a multiple of seq_len;
+ * cache_rows 0 or >= seq_len; at least one of rotate and a cache layout.
+ * workspace: >= star_linear_rope_workspace_bytes(seq_len, head_dim, rotate)
+ * bytes, 256-byte aligned, zero-filled once: the status word, then (rotate)
+ * the call's fp32 cos/sin table of its seq_len positions, built by a small
+ * kernel the call launches before the GEMM. Operands and errors as
+ * star_linear.
+ */
+size_t star_linear_rope_workspace_bytes(int seq_len, int head_dim, int rotate);
+star_status star_linear_rope(const void* x, const void* w, void* y, int M, int N, int K,
+                             int head_dim, int rotate, int seq_len, int64_t pos0, double theta,
+                             int cache_rows, void* workspace, size_t workspace_bytes,
+                             void* cuda_stream);
 
 /*
  * star_device_status — synchronises `cuda_stream`, then reads the status

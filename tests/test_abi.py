@@ -93,9 +93,18 @@ def _chunk_scratch(B, T, Hq, Hkv, D, Lcap, b):
     for n in range(1, Lcap // b + 1):
         ns = _subsplits(B, Hq, Hkv, T, n * b, b)
         if ns > 1:
-            rows = B * Hq * (n * ns + 1) * T
+            rows = B * Hq * (n * ns) * T  # the context sub-splits (the tail is written in place)
             best = max(best, up(rows * D * 4) + up(rows * 4))
     return best
+
+
+def _chunk_counters(B, T, Hq, Hkv, Lcap, b):
+    """Counters of the in-kernel sub-split reduction and merge: per (head
+    group, query tile) one per block of a context of up to Lcap rows, plus one."""
+    g = Hq // Hkv
+    hpc = 2 if g % 2 == 0 else 1
+    groups = B * Hkv * (g // hpc) * -(-T // 128)
+    return -(-(groups * (-(-Lcap // b) + 1) * 4) // 256) * 256
 
 
 def test_query_chunk_subsplit_rule():
@@ -116,7 +125,8 @@ def test_workspace_sizes(lib):
     chunk = lib.star_phase2_workspace_bytes(1, 128, 32, 8, 128, 16384 + 192, 4096)
     splits = -(-(16384 + 192) // 4096) + 1
     header = 256 + (-(-(8 * splits * 4) // 256)) * 256 + 256
-    assert chunk == header + 128 * 32 * 128 * 2 + _chunk_scratch(1, 128, 32, 8, 128, 16384 + 192, 4096)
+    assert chunk == header + 128 * 32 * 128 * 2 + _chunk_counters(1, 128, 32, 8, 16384 + 192, 4096) \
+        + _chunk_scratch(1, 128, 32, 8, 128, 16384 + 192, 4096)
     # decode path adds chunk scratch
     dec = lib.star_phase2_workspace_bytes(1, 1, 32, 8, 128, 16384 + 192, 4096)
     assert dec > 256 + 32 * 128 * 2
@@ -271,7 +281,42 @@ def test_stack_calls_validation(lib):
     assert lib.star_linear(NULL, FAKE, FAKE, 4, 64, 64, 0, NULL, 0, NULL) == INVALID
     assert lib.star_linear(FAKE, FAKE, FAKE, 4, 64, 64, 0, NULL, 1024, NULL) == INVALID
     assert lib.star_linear(FAKE, FAKE, FAKE, 4, 64, 64, 0, ODD, 1024, NULL) == INVALID
+    assert lib.star_linear(FAKE, FAKE, FAKE, 4, 64, 64, 0, NULL, 0, NULL) == INVALID  # no status word
+    assert lib.star_linear(FAKE, FAKE, FAKE, 4, 64, 64, 0, FAKE, 128, NULL) == INVALID
     assert lib.star_last_error()
+    # linear_rope: head_dim 64/128, whole heads, M = B * seq_len, cache rows >= seq_len
+    def lr(M=8, N=128, K=64, hd=64, rot=1, S=4, pos0=0, theta=1e4, rows=0, ws=FAKE, wsb=256):
+        return lib.star_linear_rope(FAKE, FAKE, FAKE, M, N, K, hd, rot, S, pos0, theta, rows, ws,
+                                    wsb, NULL)
+    assert lr(hd=96) == UNSUPPORTED
+    assert lr(N=96) == INVALID            # 1.5 heads of 64
+    assert lr(S=3) == INVALID             # M not a multiple of seq_len
+    assert lr(rows=3) == INVALID          # cache shorter than a sequence
+    assert lr(rot=0, rows=0) == INVALID   # nothing to do beyond star_linear
+    assert lr(rot=2) == INVALID
+    assert lr(pos0=-1) == INVALID
+    assert lr(theta=0.0) == INVALID
+    assert lr(ws=NULL, wsb=0) == INVALID
+    assert lr(wsb=256) == INVALID         # rotation needs room for the cos/sin table
+    assert lib.star_last_error()
+    # status word, then the fp32 (cos, sin) of seq_len positions x head_dim/2 frequencies
+    assert lib.star_linear_rope_workspace_bytes(4096, 128, 1) == 256 + 4096 * 64 * 8
+    assert lib.star_linear_rope_workspace_bytes(5, 64, 1) == 256 + 5 * 32 * 8
+    assert lib.star_linear_rope_workspace_bytes(4096, 128, 0) == 256
+
+
+def test_phase1_rotated_validation(lib):
+    def p1r(q=FAKE, o=FAKE, kc=FAKE, vc=FAKE, Lcap=64, lse=NULL, B=1, L=64, Hq=4, Hkv=2, D=64,
+            b=16, a=16, ws=FAKE, wsb=256):
+        return lib.star_phase1_encode_rotated(q, o, kc, vc, Lcap, lse, B, L, Hq, Hkv, D, b, a,
+                                              ws, wsb, NULL)
+    assert p1r(q=NULL) == INVALID
+    assert p1r(kc=ODD) == INVALID
+    assert p1r(a=17) == INVALID
+    assert p1r(Lcap=63) == INVALID
+    assert p1r(wsb=255) == INVALID        # the status word needs 256 bytes
+    assert p1r(D=80) == UNSUPPORTED
+    assert p1r(Hq=3) == INVALID
 
 
 def test_merge_and_rope_validation(lib):
@@ -295,6 +340,9 @@ def test_valid_call_without_device_reports_cuda_error(lib):
     assert _p1x(lib, G=0, src=NULL, pos=NULL, bounds=NULL) in (CUDA, UNSUPPORTED)
     assert _p2x(lib) in (CUDA, UNSUPPORTED)
     assert _p2x(lib, with_tail=0, k=NULL, v=NULL, qpos0=5000) in (CUDA, UNSUPPORTED)
+    assert lib.star_linear(FAKE, FAKE, FAKE, 4, 64, 64, 0, FAKE, 256, NULL) in (CUDA, UNSUPPORTED)
+    assert lib.star_phase1_encode_rotated(FAKE, FAKE, FAKE, FAKE, 64, NULL, 1, 64, 4, 2, 64, 16,
+                                          16, FAKE, 256, NULL) in (CUDA, UNSUPPORTED)
 
 
 def test_python_binding_raises_on_missing_library(tmp_path):

@@ -110,3 +110,61 @@ def test_phase1_without_lse_and_repeatable():
     o2, _, _, _ = encode(q, k, v, b, a, theta)
     torch.cuda.synchronize()
     assert torch.equal(o1, o2)  # deterministic, LSE output optional
+
+
+@pytest.mark.parametrize("name", ["tiny-gqa-2k", "llama8b-16k"])
+def test_phase1_against_unrounded_oracle(name):
+    """The oracle's default reading rounds the rotated Q/K to bf16 (the cache
+    the method keeps); the pure fp64 reading does not. Reported: the GPU's
+    max-abs against each reading and the two readings' own distance. The GPU
+    must meet the tolerances against the bf16 reading. Against the fp64
+    reading its output must still meet them. Its LSE may additionally move by
+    the rounding of the scores themselves: with q~, k~ the bf16 roundings of
+    the rotated q, k (relative error <= 2^-9 each), every score moves by at
+    most (2^-8 + 2^-18) * sum_i |q_i k_i| / sqrt(D), so the LSE of a row moves
+    by at most that over its visible keys (a row near a block start sees few
+    keys, so its LSE carries one score's rounding). That bound, computed per
+    row, is added to the LSE tolerance."""
+    from gpu_util import sample_rows
+
+    from block_sparse_long_rope_b200 import inputs
+    from block_sparse_long_rope_b200.configs import BY_NAME
+    from oracle import brute
+
+    w = BY_NAME[name]
+    q, k, v = inputs.make_context(w.B, w.L, w.Hq, w.Hkv, w.D, w.index, device="cuda")
+    o, lse, _, _ = encode(q, k, v, w.block_len, w.anchor_len, w.theta)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(5)
+    rows = sample_rows(w.L, w.block_len, rng, extra=64) if w.L > 4096 else np.arange(w.L)
+    rr = np.repeat(rows, w.Hq)
+    hh = np.tile(np.arange(w.Hq), rows.size)
+    bb = np.zeros_like(rr)
+    qc, kc_, vc_ = q.cpu(), k.cpu(), v.cpu()
+    go = to64(o)[0][rr, hh]
+    gl = to64(lse)[0][hh, rr]
+    ref = {}
+    for rnd in (True, False):
+        ro, rl, _ = orc.phase1_rows(qc, kc_, vc_, w.block_len, w.anchor_len, w.theta, bb, hh, rr,
+                                    round_qk=rnd)
+        ref[rnd] = (ro, rl)
+    d_rnd = (max_abs(go, ref[True][0]), max_abs(gl, ref[True][1]))
+    d_f64 = (max_abs(go, ref[False][0]), max_abs(gl, ref[False][1]))
+    d_readings = (max_abs(ref[True][0], ref[False][0]), max_abs(ref[True][1], ref[False][1]))
+    # per-row bound of the LSE shift that rounding the rotated q, k causes
+    g = w.Hq // w.Hkv
+    qr = np.abs(brute.rope_complex(qc[0, rows].double().numpy(), rows, w.theta))  # [R, Hq, D]
+    kr = np.abs(brute.rope_complex(kc_[0].double().numpy(), np.arange(w.L), w.theta))
+    _, rng4 = orc.phase1_ranges(w.L, w.block_len, w.anchor_len)
+    bound = np.empty(rr.size)
+    for i, (r, h) in enumerate(zip(rr, hh)):
+        ri = int(np.searchsorted(rows, r))
+        vis = np.r_[rng4[r, 0]:rng4[r, 1], rng4[r, 2]:rng4[r, 3]]
+        bound[i] = (2.0 ** -8 + 2.0 ** -18) * np.max(kr[vis, h // g] @ qr[ri, h]) / np.sqrt(w.D)
+    excess = float(np.max(np.abs(gl - ref[False][1]) - bound))
+    print(f"{name}: max-abs (o, lse) GPU vs bf16-Q/K oracle {d_rnd}, GPU vs fp64 oracle {d_f64}, "
+          f"between the two readings {d_readings}; LSE vs fp64 beyond the rounding bound "
+          f"{excess:.3g}")
+    assert d_rnd[0] <= TOL_O and d_rnd[1] <= TOL_LSE
+    assert d_f64[0] <= TOL_O
+    assert excess <= TOL_LSE

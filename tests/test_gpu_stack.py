@@ -1,7 +1,7 @@
 """GPU parity of the decoder stack around Star attention (StarStack:
-star_rmsnorm, star_linear through cuBLASLt, star_phase1_encode,
-star_phase2_attend) against the stack oracle, plus the row-wise calls on
-their own. bf16 values of magnitude above 1 (the residual stream) are
+star_rmsnorm, the library's tcgen05 GEMM in star_linear / star_linear_rope,
+star_phase1_encode_rotated, star_phase2_attend) against the stack oracle,
+plus the row-wise calls on their own. bf16 values of magnitude above 1 (the residual stream) are
 compared relative to max(1, |ref|): one bf16 ulp is 2^-8 of the value."""
 import numpy as np
 import pytest
@@ -58,7 +58,8 @@ def test_rmsnorm_matches_fp64_within_one_rounding():
     assert _rel(to64(y), ref) <= 2.0 ** -8
 
 
-@pytest.mark.parametrize("M,N,K", [(1536, 512, 512), (1000, 640, 4096), (24, 4096, 512)])
+@pytest.mark.parametrize("M,N,K", [(1536, 512, 512), (1000, 640, 4096), (24, 4096, 512),
+                                   (300, 264, 520), (2048, 4096, 4096)])
 def test_linear_product_and_residual_add(M, N, K):
     x = inputs.randn_bf16((M, K), 3)
     w = inputs.randn_bf16((N, K), 4, scale=K ** -0.5)
@@ -74,6 +75,43 @@ def test_linear_product_and_residual_add(M, N, K):
     assert float(np.max(np.abs(to64(p) - ab) / np.maximum(1.0, np.abs(ab)))) <= 2.0 ** -8
     # the residual add: the bf16 product plus y, rounded once more
     assert np.array_equal(to64(y), orc.round_bf16(to64(p) + y0.double().numpy()))
+
+
+@pytest.mark.parametrize("B,S,H,D,K,pos0", [(1, 1536, 8, 64, 512, 0), (2, 700, 4, 128, 1024, 0),
+                                            (1, 300, 3, 128, 264, 123456),
+                                            (1, 4096, 8, 128, 4096, 0)])
+def test_linear_rope_equals_linear_then_rope(B, S, H, D, K, pos0):
+    """The RoPE and cache epilogues give the bits of star_linear followed by
+    star_rope (the projection is rounded to bf16, then rotated with the
+    correctly rounded rotation), token-major or head-major into a cache."""
+    dev = "cuda"
+    theta = 5e5
+    M, N = B * S, H * D
+    x = inputs.randn_bf16((M, K), 11).to(dev)
+    w = inputs.randn_bf16((N, K), 12, scale=K ** -0.5).to(dev)
+    ws = star.alloc_workspace(star.star_linear_rope_workspace_bytes(S, D, True))
+    p = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=dev)
+    star.star_linear(x, w, p, workspace=ws)
+    ref = torch.empty_like(p)
+    star.star_rope(p, ref, theta, pos0=pos0)
+    # rotated, token-major
+    q = torch.full_like(p, float("nan"))
+    star.star_linear_rope(x, w, q, D, True, S, pos0, theta, 0, ws)
+    # rotated, and plain, into head-major caches with spare rows
+    Lcap = S + 5
+    kc = torch.full((B, H, Lcap, D), float("nan"), dtype=torch.bfloat16, device=dev)
+    vc = torch.full_like(kc, float("nan"))
+    star.star_linear_rope(x, w, kc, D, True, S, pos0, theta, Lcap, ws)
+    star.star_linear_rope(x, w, vc, D, False, S, pos0, theta, Lcap, ws)
+    star.star_device_status(ws)
+    torch.cuda.synchronize()
+    assert torch.equal(q, ref)
+    assert torch.equal(kc[:, :, :S], ref.permute(0, 2, 1, 3))
+    assert torch.equal(vc[:, :, :S], p.permute(0, 2, 1, 3))
+    assert torch.isnan(kc[:, :, S:].float()).all() and torch.isnan(vc[:, :, S:].float()).all()
+    # and against the oracle's correctly rounded rotation of the bf16 projection
+    rot = orc.rope(p.cpu(), np.arange(pos0, pos0 + S), theta, round_out=True)
+    np.testing.assert_array_equal(to64(q), rot)
 
 
 def test_stack_encode_and_steps_match_the_oracle():

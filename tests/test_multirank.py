@@ -94,3 +94,12 @@ def test_host_cpu_reports_model_and_cores():
     info = bench.host_cpu()
     assert info["host_cores"] == os.cpu_count()
     assert isinstance(info["cpu_model"], str) and info["cpu_model"]
+
+
+def test_multi_gpu_runs_default_to_the_sharded_deployment():
+    # one GPU: a single replica; several: one sequence's blocks over the ranks
+    assert bench.resolve_mode(None, 1) == "replicas"
+    assert bench.resolve_mode(None, 2) == "sharded"
+    assert bench.resolve_mode(None, 8) == "sharded"
+    assert bench.resolve_mode("replicas", 8) == "replicas"
+    assert bench.resolve_mode("sharded", 1) == "sharded"

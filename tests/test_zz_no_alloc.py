@@ -6,7 +6,7 @@ in cudaMalloc/cudaFree): its scratch lives in a fixed device array inside the
 library. This test calls it through the C ABI on two calls in a row and
 checks its partials against the fp64 oracle (the tolerances of the other
 parity tests) and against star_phase2_partial with a caller workspace (the
-same decode kernel with another chunk size, so fp32 rounding only), then
+same decode kernel with another chunk size: fp32 sums, bf16 weights), then
 reads the array's status word back through
 star_phase2_decode_static_status. The file is collected last so that a stop
 at the first failure has already run every other test; it also passes alone
@@ -27,7 +27,14 @@ pytestmark = pytest.mark.gpu
 
 TOL_O = 2e-2      # against the oracle: bf16-path tolerances of every parity test
 TOL_LSE = 1e-3
-TOL_SAME = 1e-4   # against the workspace entry point: the same kernel, fp32 rounding
+# Against the workspace entry point: the same kernel with another chunk size.
+# Its row sums (hence the LSE) are fp32, so those agree to fp32 rounding; the
+# P*V product takes P in bf16 (8 significant bits) relative to each chunk's
+# own running max, so two chunkings of one split round each weight
+# differently by up to 2^-9 relative, which on averaged N(0,1) values stays
+# well inside 2e-3.
+TOL_SAME_O = 2e-3
+TOL_SAME_LSE = 1e-5
 
 
 def _rand(shape, seed):
@@ -88,8 +95,8 @@ def test_static_scratch_decode_matches_oracle_and_workspace_entry(B, L, Hq, Hkv,
         star.star_device_status(ws2)
         assert torch.isfinite(po).all() and torch.isfinite(pl).all()
         # the same kernel with a caller workspace: fp32 rounding apart, equal
-        assert (po - po_ref).abs().max().item() <= TOL_SAME
-        assert (pl - pl_ref).abs().max().item() <= TOL_SAME
+        assert (po - po_ref).abs().max().item() <= TOL_SAME_O
+        assert (pl - pl_ref).abs().max().item() <= TOL_SAME_LSE
         # against the fp64 oracle, every (batch, head, token) and split
         bb, hh, tt = np.meshgrid(np.arange(B), np.arange(Hq), np.arange(T), indexing="ij")
         bb, hh, tt = bb.ravel(), hh.ravel(), tt.ravel()
