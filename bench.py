@@ -286,11 +286,12 @@ def pack_calls(calls, device=None, pin=False):
 
 def layer_launches(w):
     """Kernels one step of workload w launches: Phase 1 (RoPE + attention),
-    the query chunk (RoPE + attention, which reduces and merges in-kernel),
-    one decode kernel per token."""
+    the query chunk (RoPE + attention + the sub-split reduction with the
+    merge, or the merge alone), one decode kernel per token (which also
+    merges)."""
     chunk = 0
     if w.Tq > 0:
-        chunk = 1 if w.Tq * (w.Hq // w.Hkv) <= 16 else 2  # the decode kernel does it all
+        chunk = 1 if w.Tq * (w.Hq // w.Hkv) <= 16 else 3
     return 2 + chunk + w.Tdec
 
 

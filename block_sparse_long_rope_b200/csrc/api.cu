@@ -184,14 +184,7 @@ size_t chunk_scratch_bytes(int B, int T, int Hq, int Hkv, int D, int Lcap, int b
   return best;
 }
 
-// Counters of a query chunk's in-kernel reduction and merge: per (head
-// group, query tile) one per context block plus one for the splits; the
-// RoPE launch of the call clears them.
-int chunk_counter_words(int B, int T, int Hq, int Hkv, int Lcap, int block_len) {
-  const int g = Hq / Hkv, hpc = (g % 2 == 0) ? 2 : 1;
-  const long long groups = (long long)B * Hkv * (g / hpc) * ceil_div(T, 128);
-  return (int)(groups * (ceil_div(Lcap, block_len) + 1));
-}
+
 
 
 size_t decode_scratch_bytes(int B, int Hkv, int D, int Lcap, int block_len) {
@@ -494,8 +487,7 @@ size_t star_phase2_workspace_bytes(int B, int T, int Hq, int Hkv, int D, int Lca
   // in front, so query-chunk and decode calls can share one workspace
   const size_t head = decode_header_bytes(B, Hkv, Lcap, block_len) + align_up((size_t)B * T * Hq * D * 2);
   if (use_decode_path(T, Hq, Hkv)) return head + decode_scratch_bytes(B, Hkv, D, Lcap, block_len);
-  return head + align_up((size_t)chunk_counter_words(B, T, Hq, Hkv, Lcap, block_len) * sizeof(int)) +
-         chunk_scratch_bytes(B, T, Hq, Hkv, D, Lcap, block_len);
+  return head + chunk_scratch_bytes(B, T, Hq, Hkv, D, Lcap, block_len);
 }
 
 }  // extern "C"
@@ -581,14 +573,7 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   rp.pos = nullptr;
   rp.pos0 = q_pos0;
   star::rope_set_freq(rp, D, theta);
-  // query chunks: the counters of the attention kernel's in-kernel reduction
-  // and merge sit after the rotated q; the RoPE launch clears them
-  int* chunk_cnt = reinterpret_cast<int*>(ws + header + qrot_bytes);
-  const int n_cnt = decode ? 0 : chunk_counter_words(B, T, Hq, Hkv, Lcap, block_len);
-  const size_t cnt_bytes = align_up((size_t)n_cnt * sizeof(int));
   if (!decode) {
-    rp.zero = chunk_cnt;
-    rp.nzero = n_cnt;
     e = star::launch_rope(rp, with_tail ? 3 : 1, st);
     if (e != cudaSuccess) return cuda_fail(e, "rope launch");
   }
@@ -666,23 +651,18 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   ap.geom.tail_len = tail_len;
   ap.geom.tail = with_tail;
   // Blocks cut into sub-splits: the items' partials go to the workspace and
-  // the CTA completing a block reduces them into part_o; the CTA completing
-  // the last split of a (head group, query tile) merges the splits (attend).
-  // One launch after the RoPE kernel.
+  // one launch after the attention reduces them into part_o and, for attend,
+  // merges all splits in the same pass; otherwise the items write part_o
+  // directly and attend adds the plain merge.
   const int nsub = chunk_subsplits(B, Hq, Hkv, T, L, block_len, with_tail);
   ap.geom.nsub = nsub;
   ap.geom.sub_len = block_len / nsub;
   if (nsub > 1) {
     const size_t rows = (size_t)B * Hq * (n * nsub) * T;
-    uint8_t* sub = ws + header + qrot_bytes + cnt_bytes;
+    uint8_t* sub = ws + header + qrot_bytes;
     ap.sub_o = reinterpret_cast<float*>(sub);
     ap.sub_lse = reinterpret_cast<float*>(sub + align_up(rows * D * sizeof(float)));
   }
-  const int nq = ceil_div(T, 128);
-  ap.cnt_split = chunk_cnt;
-  ap.cnt_group = chunk_cnt + (size_t)ap.geom.groups() * nq * n;
-  ap.o_merged = static_cast<__nv_bfloat16*>(o_merged);
-  ap.lse_merged = o_merged ? lse_merged : nullptr;
   ap.mode = 1;
   ap.num_items = ap.geom.phase2_items();
   ap.qrows = T;
@@ -694,6 +674,20 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
   ap.scale_log2 = (float)(1.4426950408889634 / sqrt((double)D));
   e = star::launch_attn(ap, D, st);
   if (e != cudaSuccess) return cuda_fail(e, "phase-2 chunk attention launch");
+  if (nsub > 1) {
+    e = star::launch_chunk_finish(ap.sub_o, ap.sub_lse, nsub, n, with_tail, part_o, part_lse,
+                                  static_cast<__nv_bfloat16*>(o_merged), lse_merged, B, T, Hq, D,
+                                  st);
+    if (e != cudaSuccess) return cuda_fail(e, "sub-split reduce launch");
+  } else if (o_merged) {
+    star::MergeSegs segs{};
+    segs.nseg = 1;
+    segs.slots = nsplit;
+    segs.ns[0] = nsplit;
+    e = star::launch_lse_merge(part_o, part_lse, segs, static_cast<__nv_bfloat16*>(o_merged),
+                               lse_merged, B, T, Hq, D, st);
+    if (e != cudaSuccess) return cuda_fail(e, "lse merge launch");
+  }
   return ok();
 }
 

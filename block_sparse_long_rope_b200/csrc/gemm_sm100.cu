@@ -59,23 +59,34 @@ __device__ __forceinline__ void gemm_drain(uint64_t* bar, uint32_t parity, uint6
 __device__ __forceinline__ uint32_t bf16_bits_rn(float x) { return pack_bf16x2(x, 0.f) & 0xFFFFu; }
 __device__ __forceinline__ float bf16_round(float x) { return __uint_as_float(bf16_bits_rn(x) << 16); }
 
-// Address of output element (m, n): row-major [M, N] (cache_rows == 0) or
-// the head-major cache [B, N / hd, cache_rows, hd].
-__device__ __forceinline__ __nv_bfloat16* out_ptr(const GemmParams& p, int m, int n) {
-  if (p.cache_rows == 0) return p.y + static_cast<size_t>(m) * p.N + n;
+// Where one output row goes: element n of row m is at row + n (row-major
+// [M, N], cache_rows == 0), or at row + (n / hd) * head_stride + n % hd (the
+// head-major cache [B, N / hd, cache_rows, hd]).
+struct OutRow {
+  __nv_bfloat16* row;
+  size_t head_stride;  // 0 for row-major
+};
+__device__ __forceinline__ OutRow out_row(const GemmParams& p, int m) {
+  if (p.cache_rows == 0) return OutRow{p.y + static_cast<size_t>(m) * p.N, 0};
   const int b = m / p.seq_len, t = m - b * p.seq_len;
-  const int head = n / p.hd, d = n - head * p.hd;
-  return p.y + ((static_cast<size_t>(b) * (p.N / p.hd) + head) * p.cache_rows + t) * p.hd + d;
+  const size_t hs = static_cast<size_t>(p.cache_rows) * p.hd;
+  return OutRow{p.y + static_cast<size_t>(b) * (p.N / p.hd) * hs + static_cast<size_t>(t) * p.hd, hs};
+}
+// 8 consecutive columns from n never straddle a head (hd is a multiple of 8)
+__device__ __forceinline__ __nv_bfloat16* out_at(const GemmParams& p, const OutRow& o, int n) {
+  if (o.head_stride == 0) return o.row + n;
+  const int head = n / p.hd;
+  return o.row + head * o.head_stride + (n - head * p.hd);
 }
 
 // 32 accumulator columns of one row -> bf16 (plus the residual), stored as
 // four 16-byte vectors starting at column n (a vector past N is skipped).
-__device__ __forceinline__ void store_plain32(const GemmParams& p, int m, int n,
+__device__ __forceinline__ void store_plain32(const GemmParams& p, const OutRow& o, int n,
                                               const uint32_t (&r)[32]) {
 #pragma unroll
   for (int v = 0; v < 4; ++v) {
     if (n + 8 * v >= p.N) break;
-    __nv_bfloat16* dst = out_ptr(p, m, n + 8 * v);
+    __nv_bfloat16* dst = out_at(p, o, n + 8 * v);
     uint32_t w[4];
     if (p.accumulate) {
       const uint4 old = *reinterpret_cast<const uint4*>(dst);
@@ -96,10 +107,11 @@ __device__ __forceinline__ void store_plain32(const GemmParams& p, int m, int n,
 }
 
 // 32 bf16 values (bits in the low 16 of each word) to four 16-byte vectors at column n.
-__device__ __forceinline__ void store_bits32(const GemmParams& p, int m, int n, const uint32_t (&h)[32]) {
+__device__ __forceinline__ void store_bits32(const GemmParams& p, const OutRow& o, int n,
+                                             const uint32_t (&h)[32]) {
 #pragma unroll
   for (int v = 0; v < 4; ++v) {
-    __nv_bfloat16* dst = out_ptr(p, m, n + 8 * v);
+    __nv_bfloat16* dst = out_at(p, o, n + 8 * v);
     uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) w[j] = h[8 * v + 2 * j] | (h[8 * v + 2 * j + 1] << 16);
@@ -220,6 +232,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       const int m0 = (tile / p.n_tiles) * kBM, n0 = (tile % p.n_tiles) * kBN;
       const int m = m0 + row;
       const bool mvalid = m < p.M;
+      const OutRow orow = out_row(p, mvalid ? m : 0);
       const uint32_t tb = tmem + (static_cast<uint32_t>(32 * quad) << 16) + ab * kAccCols;
       if constexpr (RD == 0) {
 #pragma unroll 1
@@ -228,7 +241,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           tmem_ld32(tb + 32 * c, r);
           tmem_wait_ld();
           reg_fence32(r);
-          if (mvalid && n0 + 32 * c < p.N) store_plain32(p, m, n0 + 32 * c, r);
+          if (mvalid && n0 + 32 * c < p.N) store_plain32(p, orow, n0 + 32 * c, r);
         }
       } else {
         // heads of RD columns; pair (i, i + RD/2); 32 frequencies at a time,
@@ -269,8 +282,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
                 x[j] = pr & 0xFFFFu;
                 y[j] = pr >> 16;
               }
-              store_bits32(p, m, n0 + col, x);
-              store_bits32(p, m, n0 + col + RD / 2, y);
+              store_bits32(p, orow, n0 + col, x);
+              store_bits32(p, orow, n0 + col + RD / 2, y);
             }
           }
         }

@@ -138,6 +138,118 @@ __global__ void debug_wait_probe_kernel(int* status, unsigned long long limit_ns
   __syncthreads();
 }
 
+// One warp per (batch, head, token) row, lanes over D. Pass 1 reads the
+// sub-split LSEs: each block's own max m_s and sum z_s = sum_k e^(l_k - m_s)
+// give its LSE m_s + log z_s; the tail split's LSE is read as written. Pass 2
+// reads every sub-split output once: a block's partial is
+// sum_k e^(l_k - m_s) o_k / z_s (written to part_o), and the merged row adds
+// every split with weight e^(lse_s - M), M the max over the splits
+// [pith 2WVXFXZ2, minor comment on Algorithm 2]. Fixed order, deterministic.
+template <int D>
+__global__ void __launch_bounds__(256) chunk_finish_kernel(
+    const float* __restrict__ sub_o, const float* __restrict__ sub_lse, int nsub, int n, int tail,
+    float* __restrict__ part_o, float* __restrict__ part_lse, __nv_bfloat16* __restrict__ o,
+    float* __restrict__ lse, int B, int T, int Hq) {
+  constexpr int kPer = D / 32;
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
+  const int lane = threadIdx.x % 32;
+  if (warp >= B * Hq * T) return;
+  const int t = warp % T;
+  const size_t bh = static_cast<size_t>(warp / T);
+  const int nsplit = n + tail;
+  auto srow = [&](int s, int k) { return (bh * (static_cast<size_t>(n) * nsub) + s * nsub + k) * T + t; };
+  auto prow = [&](int s) { return (bh * nsplit + s) * T + t; };
+  // a block's LSE from its sub-splits (every lane computes the same value)
+  auto block_lse = [&](int s) {
+    float m = -INFINITY;
+    for (int k = 0; k < nsub; ++k) m = fmaxf(m, sub_lse[srow(s, k)]);
+    float z = 0.f;
+    if (m != -INFINITY)
+      for (int k = 0; k < nsub; ++k) {
+        const float l = sub_lse[srow(s, k)];
+        z += (l == -INFINITY) ? 0.f : expf(l - m);
+      }
+    return (z > 0.f) ? m + logf(z) : -INFINITY;
+  };
+  // pass 1: the max over the splits
+  float M = -INFINITY;
+  for (int s = 0; s < n; ++s) M = fmaxf(M, block_lse(s));
+  const float ltail = tail ? part_lse[prow(n)] : -INFINITY;
+  M = fmaxf(M, ltail);
+  // pass 2: block partials, and the merged row
+  float acc[kPer];
+#pragma unroll
+  for (int j = 0; j < kPer; ++j) acc[j] = 0.f;
+  float zm = 0.f;
+  for (int s = 0; s < n; ++s) {
+    const float ls = block_lse(s);
+    if (lane == 0) part_lse[prow(s)] = ls;
+    float bo[kPer];
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) bo[j] = 0.f;
+    if (ls != -INFINITY) {
+      for (int k = 0; k < nsub; ++k) {
+        const float l = sub_lse[srow(s, k)];
+        const float w = (l == -INFINITY) ? 0.f : expf(l - ls);  // already normalised by z_s
+        const float* src = sub_o + srow(s, k) * D + lane * kPer;
+        if constexpr (kPer == 4) {
+          const float4 v = *reinterpret_cast<const float4*>(src);
+          bo[0] += w * v.x;
+          bo[1] += w * v.y;
+          bo[2] += w * v.z;
+          bo[3] += w * v.w;
+        } else {
+          const float2 v = *reinterpret_cast<const float2*>(src);
+          bo[0] += w * v.x;
+          bo[1] += w * v.y;
+        }
+      }
+    }
+    float* dst = part_o + prow(s) * D + lane * kPer;
+    if constexpr (kPer == 4)
+      *reinterpret_cast<float4*>(dst) = make_float4(bo[0], bo[1], bo[2], bo[3]);
+    else
+      *reinterpret_cast<float2*>(dst) = make_float2(bo[0], bo[1]);
+    if (o != nullptr && M != -INFINITY && ls != -INFINITY) {
+      const float w = expf(ls - M);
+      zm += w;
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) acc[j] += w * bo[j];
+    }
+  }
+  if (o == nullptr) return;
+  if (tail && M != -INFINITY && ltail != -INFINITY) {
+    const float w = expf(ltail - M);
+    zm += w;
+    const float* src = part_o + prow(n) * D + lane * kPer;
+#pragma unroll
+    for (int j = 0; j < kPer; ++j) acc[j] += w * src[j];
+  }
+  const float inv = (zm > 0.f) ? 1.f / zm : 0.f;
+  const int b = static_cast<int>(bh / Hq), h = static_cast<int>(bh % Hq);
+  __nv_bfloat16* od = o + ((static_cast<size_t>(b) * T + t) * Hq + h) * D + lane * kPer;
+#pragma unroll
+  for (int j = 0; j < kPer; j += 2)
+    *reinterpret_cast<uint32_t*>(od + j) = pack_bf16x2(acc[j] * inv, acc[j + 1] * inv);
+  if (lse != nullptr && lane == 0) lse[bh * T + t] = (zm > 0.f) ? M + logf(zm) : -INFINITY;
+}
+
+cudaError_t launch_chunk_finish(const float* sub_o, const float* sub_lse, int nsub, int n,
+                                int tail, float* part_o, float* part_lse, __nv_bfloat16* o,
+                                float* lse, int B, int T, int Hq, int D, cudaStream_t stream) {
+  const long long rows = static_cast<long long>(B) * Hq * T;
+  if (rows == 0) return cudaSuccess;
+  const int threads = 256;
+  const unsigned blocks = static_cast<unsigned>((rows * 32 + threads - 1) / threads);
+  if (D == 128)
+    chunk_finish_kernel<128><<<blocks, threads, 0, stream>>>(sub_o, sub_lse, nsub, n, tail, part_o,
+                                                             part_lse, o, lse, B, T, Hq);
+  else
+    chunk_finish_kernel<64><<<blocks, threads, 0, stream>>>(sub_o, sub_lse, nsub, n, tail, part_o,
+                                                            part_lse, o, lse, B, T, Hq);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_debug_wait_probe(int* status, unsigned long long limit_ns, cudaStream_t stream) {
   debug_wait_probe_kernel<<<1, 32, 0, stream>>>(status, limit_ns);
   return cudaGetLastError();

@@ -59,12 +59,12 @@ struct AttnCfg {
 
 constexpr int kAttnThreads = 320;
 
-// ---- Phase-2 query chunks: where an item's rows go, and the in-kernel
-// sub-split reduction and split merge ----------------------------------------
+// ---- Phase-2 query chunks: where an item's rows go ---------------------------
 // An item of a block cut into sub-splits (nsub > 1) writes sub-split row
-// (b, head, split, qrow) of sub_o / sub_lse; any other item (a whole block,
-// or the tail) writes its split's row of part_o / part_lse directly. Returns
-// the row index; *to_sub tells which pair of buffers it indexes.
+// (b, head, split, qrow) of sub_o / sub_lse (chunk_finish_kernel reduces
+// them); any other item (a whole block, or the tail) writes its split's row
+// of part_o / part_lse directly. Returns the row index; *to_sub tells which
+// pair of buffers it indexes.
 __device__ __forceinline__ size_t p2_row(const AttnParams& p, const WorkItem& w, int head, int qrow,
                                          bool* to_sub) {
   const AttnGeom& g = p.geom;
@@ -75,138 +75,6 @@ __device__ __forceinline__ size_t p2_row(const AttnParams& p, const WorkItem& w,
   return (bh * p.nsplit + api) * g.T + qrow;
 }
 
-// Exact LSE merge of `cnt` partial rows (row(k) indexes lse / o) into one
-// output row: m = max lse_k, w_k = e^(lse_k - m), o = sum w_k o_k / sum w_k,
-// lse = m + log sum w_k, in fixed order [pith 2WVXFXZ2, minor comment on
-// Algorithm 2]. Eight lanes (a quarter warp) take one row, so a warp merges
-// four rows at once; a lane covers D/8 floats as float4s, and the loads of
-// several partials (16 float4s a lane) are issued before they are
-// accumulated. All 32 lanes call it (cnt is the same for the whole warp);
-// `active` is false for a quarter without a row. Writes fp32 (out_o) or bf16
-// (out_b) and the LSE (out_lse, nullable).
-template <int D, typename RowAt>
-__device__ __forceinline__ void merge_rows(int cnt, RowAt row, bool active, const float* lse,
-                                           const float* o, float* out_o, __nv_bfloat16* out_b,
-                                           float* out_lse) {
-  constexpr int kV = D / 32;          // float4s per lane
-  constexpr int kB = 16 / kV;         // partials loaded before use (16 float4s a lane)
-  const int lane = threadIdx.x & 31, q8 = lane & 7, base = lane & 24;
-  float m = -INFINITY;
-  if (active)
-    for (int k = q8; k < cnt; k += 8) m = fmaxf(m, lse[row(k)]);
-#pragma unroll
-  for (int off = 4; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-  float4 acc[kV];
-#pragma unroll
-  for (int v = 0; v < kV; ++v) acc[v] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float z = 0.f;
-  for (int k0 = 0; k0 < cnt; k0 += kB) {
-    float wl = 0.f;
-    if (active && q8 < kB && k0 + q8 < cnt && m != -INFINITY) {
-      const float l = lse[row(k0 + q8)];
-      wl = (l == -INFINITY) ? 0.f : expf(l - m);
-    }
-    float zs = wl;
-#pragma unroll
-    for (int off = 4; off > 0; off >>= 1) zs += __shfl_xor_sync(0xffffffffu, zs, off);
-    z += zs;
-    float4 x[kB][kV];
-#pragma unroll
-    for (int j = 0; j < kB; ++j) {
-      if (active && k0 + j < cnt) {
-        const float4* src = reinterpret_cast<const float4*>(o + row(k0 + j) * D);
-#pragma unroll
-        for (int v = 0; v < kV; ++v) x[j][v] = src[q8 + 8 * v];
-      }
-    }
-#pragma unroll
-    for (int j = 0; j < kB; ++j) {
-      const float w = __shfl_sync(0xffffffffu, wl, base + j);
-      if (active && k0 + j < cnt) {
-#pragma unroll
-        for (int v = 0; v < kV; ++v) {
-          acc[v].x += w * x[j][v].x;
-          acc[v].y += w * x[j][v].y;
-          acc[v].z += w * x[j][v].z;
-          acc[v].w += w * x[j][v].w;
-        }
-      }
-    }
-  }
-  if (!active) return;
-  const float inv = (z > 0.f) ? 1.f / z : 0.f;
-#pragma unroll
-  for (int v = 0; v < kV; ++v) {
-    const float4 r = make_float4(acc[v].x * inv, acc[v].y * inv, acc[v].z * inv, acc[v].w * inv);
-    const int c = 4 * (q8 + 8 * v);
-    if (out_o) *reinterpret_cast<float4*>(out_o + c) = r;
-    if (out_b) {
-      uint2 pk;
-      pk.x = pack_bf16x2(r.x, r.y);
-      pk.y = pack_bf16x2(r.z, r.w);
-      *reinterpret_cast<uint2*>(out_b + c) = pk;
-    }
-  }
-  if (out_lse && q8 == 0) *out_lse = (z > 0.f) ? m + logf(z) : -INFINITY;
-}
-
-// Publishes this CTA's writes and counts it in; true for the last of
-// `count` arrivals, after which the others' writes are visible. Every thread
-// of the CTA calls it; one thread touches the counter.
-__device__ __forceinline__ bool count_in_last(int* counter, int count) {
-  __shared__ int s_last;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    s_last = atomicAdd(counter, 1) == count - 1;
-    __threadfence();
-  }
-  __syncthreads();
-  return s_last != 0;
-}
-
-// After a query-chunk item has written its rows: the CTA that completes a
-// block's sub-splits reduces them into the block's split partial; the CTA
-// that completes the last split of a (head group, query tile) merges all
-// splits into o_merged / lse_merged (when asked). All threads of the CTA.
-template <int D>
-__device__ void query_chunk_fold(const AttnParams& p) {
-  const AttnGeom& g = p.geom;
-  const WorkItem w = g.phase2_item(blockIdx.x);  // recomputed: nothing stays live across the loop
-  const int G = g.groups(), nq = g.phase2_qtiles();
-  const int rem = blockIdx.x % (nq * G);
-  const int gq = (rem % G) * nq + rem / G;  // (group, query tile)
-  const int warp = threadIdx.x >> 5, quarter = (threadIdx.x & 31) >> 3;
-  constexpr int kQuarters = kAttnThreads / 8;  // rows merged at once by the CTA
-  const int rows = w.q_hi - w.q_lo, hpc = g.hpc, pairs = rows * hpc;
-  const bool sub = g.nsub > 1 && w.split < g.n * g.nsub;
-  if (sub) {
-    const int blk = w.split / g.nsub;
-    if (!count_in_last(&p.cnt_split[gq * g.n + blk], g.nsub)) return;
-    for (int p0 = 0; p0 < pairs; p0 += kQuarters) {  // warp-uniform trip count
-      const int pr = p0 + 4 * warp + quarter;
-      const bool active = pr < pairs;
-      const int head = w.slot0 + (active ? pr / rows : 0), qrow = w.q_lo + (active ? pr % rows : 0);
-      const size_t bh = static_cast<size_t>(w.b) * g.Hq + head;
-      const size_t s0 = (bh * (g.n * g.nsub) + blk * g.nsub) * g.T + qrow;
-      const size_t out = (bh * p.nsplit + blk) * g.T + qrow;
-      merge_rows<D>(g.nsub, [&](int k) { return s0 + static_cast<size_t>(k) * g.T; }, active,
-                    p.sub_lse, p.sub_o, p.part_o + out * D, nullptr, p.part_lse + out);
-    }
-  }
-  if (p.o_merged == nullptr) return;
-  if (!count_in_last(&p.cnt_group[gq], p.nsplit)) return;
-  for (int p0 = 0; p0 < pairs; p0 += kQuarters) {
-    const int pr = p0 + 4 * warp + quarter;
-    const bool active = pr < pairs;
-    const int head = w.slot0 + (active ? pr / rows : 0), qrow = w.q_lo + (active ? pr % rows : 0);
-    const size_t bh = static_cast<size_t>(w.b) * g.Hq + head;
-    __nv_bfloat16* ob = p.o_merged + ((static_cast<size_t>(w.b) * g.T + qrow) * g.Hq + head) * D;
-    float* lo = p.lse_merged ? p.lse_merged + bh * g.T + qrow : nullptr;
-    merge_rows<D>(p.nsplit, [&](int k) { return (bh * p.nsplit + k) * g.T + qrow; }, active,
-                  p.part_lse, p.part_o, nullptr, ob, lo);
-  }
-}
 constexpr uint64_t kDrainNs = 100000000ull;  // 100 ms
 
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
@@ -571,9 +439,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
   __syncthreads();
   tc_fence_after();
   if (warp == 9) tmem_dealloc(tmem, C::kTmemCols);
-  if constexpr (kMode == 1) {
-    if (!abort_flag) query_chunk_fold<D>(p);
-  }
 }
 
 size_t attn_smem_bytes(int D) {

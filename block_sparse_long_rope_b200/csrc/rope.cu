@@ -25,8 +25,7 @@
 // sequences, fewer for a handful of new tokens so that the grid still fills
 // the GPU); it first computes the (cos, sin) table of its tokens in shared
 // memory, then streams 16-byte vectors: a thread rotates chunk c of the first
-// half together with chunk c of the second half of one head. A launch can
-// also clear a few counters of the kernel that follows it (p.zero).
+// half together with chunk c of the second half of one head.
 #include <cmath>
 
 #include "rope_math.cuh"
@@ -43,11 +42,6 @@ template <int D>
 __global__ void __launch_bounds__(kRopeThreads) rope_kernel(const __grid_constant__ RopeParams p) {
   constexpr int kHalf = D / 2, kCpr = kHalf / 8;  // 16-byte chunks per half row
   const RopeJob& job = p.job[blockIdx.z];
-  if (p.zero) {  // counters of the next kernel in the stream
-    const int cta = blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z);
-    const int nthr = gridDim.x * gridDim.y * gridDim.z * kRopeThreads;
-    for (int i = cta * kRopeThreads + threadIdx.x; i < p.nzero; i += nthr) p.zero[i] = 0;
-  }
   const int tok0 = blockIdx.x * p.tpc;
   const int b = blockIdx.y;
   const int ntok = imin(p.tpc, p.S - tok0);

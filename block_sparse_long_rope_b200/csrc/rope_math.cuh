@@ -86,12 +86,34 @@ __device__ __forceinline__ uint32_t rope_rotate_pair_bf16(float a, float b, floa
   });
 }
 
-// As above with the fp64 cos/sin of pos * inv_freq recomputed on the rare
-// slow path (c32/s32 must be the fp32 roundings of rope_angle's results).
+// The rare slow path of rope_rotate_pair_bf16_at, kept out of line so that
+// unrolled callers stay small: recomputes the fp64 cos/sin of pos * inv_freq
+// and rounds the outputs flagged in `need` (bit 0: first, bit 1: second)
+// exactly as rope_rotate_pair_bf16_with does; `fast` holds the others.
+static __device__ __noinline__ uint32_t rope_pair_exact_at(float a, float b, long long pos,
+                                                    double inv_freq, uint32_t fast, uint32_t need) {
+  double cd, sd;
+  rope_angle(pos, inv_freq, &cd, &sd);
+  const double ad = a, bd = b;
+  uint32_t o0 = fast & 0xFFFFu, o1 = fast >> 16;
+  if (need & 1u) o0 = pack_bf16x2(f32_round_odd(ad * cd - bd * sd), 0.f) & 0xFFFFu;
+  if (need & 2u) o1 = pack_bf16x2(f32_round_odd(bd * cd + ad * sd), 0.f) & 0xFFFFu;
+  return o0 | (o1 << 16);
+}
+
+// As rope_rotate_pair_bf16_with, with the fp64 cos/sin of pos * inv_freq
+// recomputed on the rare slow path (c32/s32 must be the fp32 roundings of
+// rope_angle's results): the same bits.
 __device__ __forceinline__ uint32_t rope_rotate_pair_bf16_at(float a, float b, float c32, float s32,
                                                              long long pos, double inv_freq) {
-  return rope_rotate_pair_bf16_with(a, b, c32, s32,
-                                    [&](double* c, double* s) { rope_angle(pos, inv_freq, c, s); });
+  const float e = 2.3841858e-07f * (fabsf(a) + fabsf(b));
+  const float y0 = fmaf(a, c32, -(b * s32));
+  const float y1 = fmaf(b, c32, a * s32);
+  const uint32_t r0 = pack_bf16x2(y0 - e, y0 + e), r1 = pack_bf16x2(y1 - e, y1 + e);
+  const uint32_t o0 = r0 & 0xFFFFu, o1 = r1 & 0xFFFFu;
+  const uint32_t need = (o0 == (r0 >> 16) ? 0u : 1u) | (o1 == (r1 >> 16) ? 0u : 2u);
+  if (need) return rope_pair_exact_at(a, b, pos, inv_freq, o0 | (o1 << 16), need);
+  return o0 | (o1 << 16);
 }
 
 }  // namespace star

@@ -35,8 +35,6 @@ struct RopeParams {
   const int32_t* src;
   int nsrc, nx;
   int* status;
-  int* zero;   // nullable: nzero ints cleared by the launch (counters of the next kernel)
-  int nzero;
   double inv_freq[64];  // theta^(-2i/D), i < D/2 (fp64, from the host)
 };
 constexpr int kRopeMaxTok = 8;
@@ -65,14 +63,10 @@ struct AttnParams {
   float* part_o;     // Phase 2: [B, Hq, nsplit, T, D], nsplit = n + tail (the API's splits)
   float* part_lse;   // Phase 2: [B, Hq, nsplit, T]
   // Phase-2 query chunks whose blocks are cut into nsub sub-splits: the
-  // items' partials go to sub_o / sub_lse ([B, Hq, n * nsub, T, D] / [.., T]);
-  // the CTA finishing a block's last sub-split reduces them into part_o.
+  // items' partials go to sub_o / sub_lse ([B, Hq, n * nsub, T, D] / [.., T]),
+  // which launch_chunk_finish reduces into part_o.
   float* sub_o;
   float* sub_lse;
-  int* cnt_split;    // [groups, qtiles, n] finished sub-splits (cleared by the RoPE launch)
-  int* cnt_group;    // [groups, qtiles] finished splits (cleared by the RoPE launch)
-  __nv_bfloat16* o_merged;  // nullable: [B, T, Hq, D]; the CTA finishing the last split merges
-  float* lse_merged;        // nullable: [B, Hq, T]
   int* status;
   float scale_log2;  // log2(e) / sqrt(D)
   float scale_ln;    // 1 / sqrt(D)
@@ -129,6 +123,14 @@ struct MergeSegs {
 cudaError_t launch_lse_merge(const float* part_o, const float* part_lse, const MergeSegs& segs,
                              __nv_bfloat16* o, float* lse, int B, int T, int Hq, int D,
                              cudaStream_t stream);
+// After a query chunk whose n context blocks were cut into nsub sub-splits
+// (sub_o / sub_lse [B, Hq, n * nsub, T, D] / [.., T]): reduces each block's
+// sub-splits into part_o / part_lse [B, Hq, n + tail, T, (D)] (the tail
+// split is already there) and, when o is not NULL, merges all n + tail
+// splits into o [B, T, Hq, D] / lse [B, Hq, T] in the same pass.
+cudaError_t launch_chunk_finish(const float* sub_o, const float* sub_lse, int nsub, int n,
+                                int tail, float* part_o, float* part_lse, __nv_bfloat16* o,
+                                float* lse, int B, int T, int Hq, int D, cudaStream_t stream);
 
 // ---- projection GEMM (tcgen05): y[M, N] = x[M, K] w[N, K]^T with epilogues --
 struct GemmParams {

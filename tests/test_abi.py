@@ -98,15 +98,6 @@ def _chunk_scratch(B, T, Hq, Hkv, D, Lcap, b):
     return best
 
 
-def _chunk_counters(B, T, Hq, Hkv, Lcap, b):
-    """Counters of the in-kernel sub-split reduction and merge: per (head
-    group, query tile) one per block of a context of up to Lcap rows, plus one."""
-    g = Hq // Hkv
-    hpc = 2 if g % 2 == 0 else 1
-    groups = B * Hkv * (g // hpc) * -(-T // 128)
-    return -(-(groups * (-(-Lcap // b) + 1) * 4) // 256) * 256
-
-
 def test_query_chunk_subsplit_rule():
     # llama8b-16k query chunk: 80 items -> 2 sub-splits per block, 144 items
     assert _subsplits(1, 32, 8, 128, 16384, 4096) == 2
@@ -125,8 +116,7 @@ def test_workspace_sizes(lib):
     chunk = lib.star_phase2_workspace_bytes(1, 128, 32, 8, 128, 16384 + 192, 4096)
     splits = -(-(16384 + 192) // 4096) + 1
     header = 256 + (-(-(8 * splits * 4) // 256)) * 256 + 256
-    assert chunk == header + 128 * 32 * 128 * 2 + _chunk_counters(1, 128, 32, 8, 16384 + 192, 4096) \
-        + _chunk_scratch(1, 128, 32, 8, 128, 16384 + 192, 4096)
+    assert chunk == header + 128 * 32 * 128 * 2 + _chunk_scratch(1, 128, 32, 8, 128, 16384 + 192, 4096)
     # decode path adds chunk scratch
     dec = lib.star_phase2_workspace_bytes(1, 1, 32, 8, 128, 16384 + 192, 4096)
     assert dec > 256 + 32 * 128 * 2
