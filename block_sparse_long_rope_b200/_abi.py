@@ -41,6 +41,7 @@ EXPORTS = (
     "star_linear",
     "star_linear_rope",
     "star_linear_rope_workspace_bytes",
+    "star_linear_kv_cache",
     "star_device_status",
     "star_debug_index",
     "star_debug_wait_probe",
@@ -98,6 +99,9 @@ def load(path: str = LIB_PATH):
                                                    _I, _P, _SZ, _P]
         lib.star_linear_rope_workspace_bytes.restype = _SZ
         lib.star_linear_rope_workspace_bytes.argtypes = [_I, _I, _I]
+        lib.star_linear_kv_cache.restype = _I
+        lib.star_linear_kv_cache.argtypes = [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I64, _D, _I, _P,
+                                             _SZ, _P]
         lib.star_linear_rope.restype = _I
         lib.star_linear_rope.argtypes = [_P, _P, _P, _I, _I, _I, _I, _I, _I, _I64, _D, _I, _P,
                                          _SZ, _P]

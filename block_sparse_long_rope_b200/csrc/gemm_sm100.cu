@@ -66,11 +66,12 @@ struct OutRow {
   __nv_bfloat16* row;
   size_t head_stride;  // 0 for row-major
 };
-__device__ __forceinline__ OutRow out_row(const GemmParams& p, int m) {
-  if (p.cache_rows == 0) return OutRow{p.y + static_cast<size_t>(m) * p.N, 0};
+// Output row m of buffer y (width nw columns, in heads of hd for the cache).
+__device__ __forceinline__ OutRow out_row(const GemmParams& p, __nv_bfloat16* y, int nw, int m) {
+  if (p.cache_rows == 0) return OutRow{y + static_cast<size_t>(m) * nw, 0};
   const int b = m / p.seq_len, t = m - b * p.seq_len;
   const size_t hs = static_cast<size_t>(p.cache_rows) * p.hd;
-  return OutRow{p.y + static_cast<size_t>(b) * (p.N / p.hd) * hs + static_cast<size_t>(t) * p.hd, hs};
+  return OutRow{y + static_cast<size_t>(b) * (nw / p.hd) * hs + static_cast<size_t>(t) * p.hd, hs};
 }
 // 8 consecutive columns from n never straddle a head (hd is a multiple of 8)
 __device__ __forceinline__ __nv_bfloat16* out_at(const GemmParams& p, const OutRow& o, int n) {
@@ -232,7 +233,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       const int m0 = (tile / p.n_tiles) * kBM, n0 = (tile % p.n_tiles) * kBN;
       const int m = m0 + row;
       const bool mvalid = m < p.M;
-      const OutRow orow = out_row(p, mvalid ? m : 0);
+      const OutRow orow = out_row(p, p.y, p.n_split, mvalid ? m : 0);
+      const OutRow orow2 = out_row(p, p.y2, p.N - p.n_split, mvalid ? m : 0);
       const uint32_t tb = tmem + (static_cast<uint32_t>(32 * quad) << 16) + ab * kAccCols;
       if constexpr (RD == 0) {
 #pragma unroll 1
@@ -271,6 +273,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             tmem_wait_ld();
             reg_fence32(x);
             reg_fence32(y);
+            if (n0 + h * RD >= p.n_split) {  // a V head of a K/V projection: no rotation
+              if (mvalid) {
+                store_plain32(p, orow2, n0 + col - p.n_split, x);
+                store_plain32(p, orow2, n0 + col + RD / 2 - p.n_split, y);
+              }
+              continue;
+            }
             if (mvalid) {
 #pragma unroll
               for (int j = 0; j < 32; ++j) {

@@ -138,12 +138,13 @@ __global__ void debug_wait_probe_kernel(int* status, unsigned long long limit_ns
   __syncthreads();
 }
 
-// One warp per (batch, head, token) row, lanes over D. Pass 1 reads the
-// sub-split LSEs: each block's own max m_s and sum z_s = sum_k e^(l_k - m_s)
-// give its LSE m_s + log z_s; the tail split's LSE is read as written. Pass 2
-// reads every sub-split output once: a block's partial is
-// sum_k e^(l_k - m_s) o_k / z_s (written to part_o), and the merged row adds
-// every split with weight e^(lse_s - M), M the max over the splits
+// One warp per (batch, head, token) row, lanes over D. Pass 1 (lanes over
+// blocks): lane s takes block s's sub-split LSEs, its max m_s and sum
+// z_s = sum_k e^(l_k - m_s), hence its LSE m_s + log z_s; the tail split's
+// LSE is read as written; M is the max over the splits. Pass 2 (lanes over
+// D) reads every sub-split output once, four blocks' rows issued before they
+// are used: a block's partial is sum_k e^(l_k - lse_s) o_k (written to
+// part_o), and the merged row adds every split with weight e^(lse_s - M)
 // [pith 2WVXFXZ2, minor comment on Algorithm 2]. Fixed order, deterministic.
 template <int D>
 __global__ void __launch_bounds__(256) chunk_finish_kernel(
@@ -151,6 +152,8 @@ __global__ void __launch_bounds__(256) chunk_finish_kernel(
     float* __restrict__ part_o, float* __restrict__ part_lse, __nv_bfloat16* __restrict__ o,
     float* __restrict__ lse, int B, int T, int Hq) {
   constexpr int kPer = D / 32;
+  constexpr int kMaxSub = 4;   // sub-splits per block (the cut rule makes at most 4)
+  constexpr int kBlk = 4;      // blocks whose rows are loaded together
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
   if (warp >= B * Hq * T) return;
@@ -159,71 +162,98 @@ __global__ void __launch_bounds__(256) chunk_finish_kernel(
   const int nsplit = n + tail;
   auto srow = [&](int s, int k) { return (bh * (static_cast<size_t>(n) * nsub) + s * nsub + k) * T + t; };
   auto prow = [&](int s) { return (bh * nsplit + s) * T + t; };
-  // a block's LSE from its sub-splits (every lane computes the same value)
-  auto block_lse = [&](int s) {
-    float m = -INFINITY;
-    for (int k = 0; k < nsub; ++k) m = fmaxf(m, sub_lse[srow(s, k)]);
+  auto block_lse = [&](int s) {  // lse of block s from its sub-splits
+    float l[kMaxSub], m = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kMaxSub; ++k) {
+      l[k] = (k < nsub) ? sub_lse[srow(s, k)] : -INFINITY;
+      m = fmaxf(m, l[k]);
+    }
     float z = 0.f;
-    if (m != -INFINITY)
-      for (int k = 0; k < nsub; ++k) {
-        const float l = sub_lse[srow(s, k)];
-        z += (l == -INFINITY) ? 0.f : expf(l - m);
-      }
+#pragma unroll
+    for (int k = 0; k < kMaxSub; ++k) z += (l[k] == -INFINITY) ? 0.f : expf(l[k] - m);
     return (z > 0.f) ? m + logf(z) : -INFINITY;
   };
-  // pass 1: the max over the splits
-  float M = -INFINITY;
-  for (int s = 0; s < n; ++s) M = fmaxf(M, block_lse(s));
-  const float ltail = tail ? part_lse[prow(n)] : -INFINITY;
-  M = fmaxf(M, ltail);
+  // pass 1: block LSEs (lane s holds block s of each 32-block round), the max
+  float M = tail ? part_lse[prow(n)] : -INFINITY;
+  for (int s0 = 0; s0 < n; s0 += 32) {
+    const int s = s0 + lane;
+    const float ls = (s < n) ? block_lse(s) : -INFINITY;
+    if (s < n) part_lse[prow(s)] = ls;
+    M = fmaxf(M, ls);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
   // pass 2: block partials, and the merged row
   float acc[kPer];
 #pragma unroll
   for (int j = 0; j < kPer; ++j) acc[j] = 0.f;
   float zm = 0.f;
-  for (int s = 0; s < n; ++s) {
-    const float ls = block_lse(s);
-    if (lane == 0) part_lse[prow(s)] = ls;
-    float bo[kPer];
+  for (int s0 = 0; s0 < n; s0 += kBlk) {
+    float lsb[kBlk], w[kBlk][kMaxSub];
+    float4 v[kBlk][kMaxSub][1];  // D = 128: a float4 per lane
+    float2 v2[kBlk][kMaxSub];    // D = 64: a float2 per lane
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) bo[j] = 0.f;
-    if (ls != -INFINITY) {
-      for (int k = 0; k < nsub; ++k) {
-        const float l = sub_lse[srow(s, k)];
-        const float w = (l == -INFINITY) ? 0.f : expf(l - ls);  // already normalised by z_s
-        const float* src = sub_o + srow(s, k) * D + lane * kPer;
-        if constexpr (kPer == 4) {
-          const float4 v = *reinterpret_cast<const float4*>(src);
-          bo[0] += w * v.x;
-          bo[1] += w * v.y;
-          bo[2] += w * v.z;
-          bo[3] += w * v.w;
-        } else {
-          const float2 v = *reinterpret_cast<const float2*>(src);
-          bo[0] += w * v.x;
-          bo[1] += w * v.y;
+    for (int i = 0; i < kBlk; ++i) {
+      const int s = s0 + i;
+      lsb[i] = -INFINITY;
+      if (s >= n) continue;
+      lsb[i] = block_lse(s);  // the same arithmetic as pass 1: the same value in every lane
+#pragma unroll
+      for (int k = 0; k < kMaxSub; ++k) {
+        w[i][k] = 0.f;
+        if (k < nsub && lsb[i] != -INFINITY) {
+          const float l = sub_lse[srow(s, k)];
+          w[i][k] = (l == -INFINITY) ? 0.f : expf(l - lsb[i]);
+          const float* src = sub_o + srow(s, k) * D + lane * kPer;
+          if constexpr (kPer == 4) v[i][k][0] = *reinterpret_cast<const float4*>(src);
+          else v2[i][k] = *reinterpret_cast<const float2*>(src);
         }
       }
     }
-    float* dst = part_o + prow(s) * D + lane * kPer;
-    if constexpr (kPer == 4)
-      *reinterpret_cast<float4*>(dst) = make_float4(bo[0], bo[1], bo[2], bo[3]);
-    else
-      *reinterpret_cast<float2*>(dst) = make_float2(bo[0], bo[1]);
-    if (o != nullptr && M != -INFINITY && ls != -INFINITY) {
-      const float w = expf(ls - M);
-      zm += w;
 #pragma unroll
-      for (int j = 0; j < kPer; ++j) acc[j] += w * bo[j];
+    for (int i = 0; i < kBlk; ++i) {
+      const int s = s0 + i;
+      if (s >= n) continue;
+      float bo[kPer];
+#pragma unroll
+      for (int j = 0; j < kPer; ++j) bo[j] = 0.f;
+#pragma unroll
+      for (int k = 0; k < kMaxSub; ++k) {
+        if (w[i][k] == 0.f) continue;
+        if constexpr (kPer == 4) {
+          bo[0] += w[i][k] * v[i][k][0].x;
+          bo[1] += w[i][k] * v[i][k][0].y;
+          bo[2] += w[i][k] * v[i][k][0].z;
+          bo[3] += w[i][k] * v[i][k][0].w;
+        } else {
+          bo[0] += w[i][k] * v2[i][k].x;
+          bo[1] += w[i][k] * v2[i][k].y;
+        }
+      }
+      float* dst = part_o + prow(s) * D + lane * kPer;
+      if constexpr (kPer == 4)
+        *reinterpret_cast<float4*>(dst) = make_float4(bo[0], bo[1], bo[2], bo[3]);
+      else
+        *reinterpret_cast<float2*>(dst) = make_float2(bo[0], bo[1]);
+      if (o != nullptr && M != -INFINITY && lsb[i] != -INFINITY) {
+        const float wm = expf(lsb[i] - M);
+        zm += wm;
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) acc[j] += wm * bo[j];
+      }
     }
   }
   if (o == nullptr) return;
-  if (tail && M != -INFINITY && ltail != -INFINITY) {
-    const float w = expf(ltail - M);
-    zm += w;
-    const float* src = part_o + prow(n) * D + lane * kPer;
+  if (tail) {
+    const float ltail = part_lse[prow(n)];
+    if (M != -INFINITY && ltail != -INFINITY) {
+      const float wt = expf(ltail - M);
+      zm += wt;
+      const float* src = part_o + prow(n) * D + lane * kPer;
 #pragma unroll
-    for (int j = 0; j < kPer; ++j) acc[j] += w * src[j];
+      for (int j = 0; j < kPer; ++j) acc[j] += wt * src[j];
+    }
   }
   const float inv = (zm > 0.f) ? 1.f / zm : 0.f;
   const int b = static_cast<int>(bh / Hq), h = static_cast<int>(bh % Hq);

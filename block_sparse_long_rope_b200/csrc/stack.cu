@@ -98,7 +98,8 @@ bool misaligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t
 // Shared body of star_linear / star_linear_rope: checks, TMA maps, launch.
 star_status run_gemm(const void* x, const void* w, void* y, int M, int N, int K, int accumulate,
                      int head_dim, int rotate, int seq_len, long long pos0, double theta,
-                     int cache_rows, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+                     int cache_rows, void* workspace, size_t workspace_bytes, void* cuda_stream,
+                     void* y2 = nullptr, int n_split = 0) {
   if (M < 1 || N < 1 || K < 1 || N % 8 || K % 8)
     return stack_fail(STAR_ERR_INVALID_ARG, "bad shape M=%d N=%d K=%d (N, K multiples of 8)", M, N, K);
   if (!x || !w || !y || misaligned(x, 16) || misaligned(w, 16) || misaligned(y, 16))
@@ -130,6 +131,8 @@ star_status run_gemm(const void* x, const void* w, void* y, int M, int N, int K,
   p.seq_len = seq_len;
   p.cache_rows = cache_rows;
   p.pos0 = pos0;
+  p.n_split = y2 ? n_split : N;
+  p.y2 = static_cast<__nv_bfloat16*>(y2 ? y2 : y);
   p.status = static_cast<int*>(workspace);
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   cudaError_t e;
@@ -210,6 +213,28 @@ star_status star_linear_rope(const void* x, const void* w, void* y, int M, int N
     return stack_fail(STAR_ERR_INVALID_ARG, "pos0 must be >= 0 and theta > 0");
   return run_gemm(x, w, y, M, N, K, 0, head_dim, rotate, seq_len, pos0, theta, cache_rows,
                   workspace, workspace_bytes, cuda_stream);
+}
+
+star_status star_linear_kv_cache(const void* x, const void* w_kv, void* k_cache, void* v_cache,
+                                 int M, int N, int K, int head_dim, int seq_len, int64_t pos0,
+                                 double theta, int cache_rows, void* workspace,
+                                 size_t workspace_bytes, void* cuda_stream) {
+  if (head_dim != 64 && head_dim != 128)
+    return stack_fail(STAR_ERR_UNSUPPORTED, "head_dim %d not supported (64 or 128)", head_dim);
+  if (N < 1 || N % head_dim)
+    return stack_fail(STAR_ERR_INVALID_ARG, "N (%d) must be whole heads of %d", N, head_dim);
+  if (seq_len < 1 || M % seq_len)
+    return stack_fail(STAR_ERR_INVALID_ARG, "M (%d) must be a multiple of seq_len (%d)", M, seq_len);
+  if (cache_rows < seq_len)
+    return stack_fail(STAR_ERR_INVALID_ARG, "cache_rows (%d) must be >= seq_len (%d)", cache_rows,
+                      seq_len);
+  if (pos0 < 0 || !(theta > 0.0))
+    return stack_fail(STAR_ERR_INVALID_ARG, "pos0 must be >= 0 and theta > 0");
+  if (!v_cache || misaligned(v_cache, 16))
+    return stack_fail(STAR_ERR_INVALID_ARG, "v_cache must be non-NULL and 16-byte aligned");
+  if ((long long)N * 2 > (1ll << 30)) return stack_fail(STAR_ERR_INVALID_ARG, "N too large");
+  return run_gemm(x, w_kv, k_cache, M, 2 * N, K, 0, head_dim, 1, seq_len, pos0, theta,
+                  cache_rows, workspace, workspace_bytes, cuda_stream, v_cache, N);
 }
 
 }  // extern "C"

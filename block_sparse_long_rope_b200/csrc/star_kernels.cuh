@@ -147,6 +147,10 @@ struct GemmParams {
   long long pos0;   // RoPE position of token t = pos0 + t
   double inv_freq[64];  // theta^(-2i/rd), i < rd/2
   const float2* rope_tab;  // [seq_len][rd/2] fp32 roundings of (cos, sin)(pos * inv_freq)
+  // K and V in one GEMM: columns n >= n_split go, unrotated, to y2 as its
+  // column n - n_split (same layout as y); n_split = N otherwise
+  int n_split;
+  __nv_bfloat16* y2;
   int* status;      // device status word (bounded waits)
 };
 size_t gemm_smem_bytes();

@@ -40,6 +40,8 @@ class StarStack:
         self.q2 = torch.empty((B * Tmax * Hq * D,), **bf)
         self.k2 = torch.empty((B * Tmax * Hkv * D,), **bf)
         self.v2 = torch.empty((B * Tmax * Hkv * D,), **bf)
+        # each layer's K and V projection weights stacked, for one K/V GEMM
+        self.w_kv = [torch.cat([wt["wk"], wt["wv"]], dim=0).contiguous() for wt in weights]
         # the GEMMs' status word and the RoPE epilogue's cos/sin table
         self.gemm_ws = star.alloc_workspace(
             star.star_linear_rope_workspace_bytes(max(L, Tmax), D, True), dev)
@@ -47,18 +49,16 @@ class StarStack:
     def encode_layer(self, x, index):
         """Phase 1 of layer `index` on the residual stream x [B, L, dm] bf16
         (updated in place); fills that layer's KV cache rows [0, L). The Q
-        projection leaves Q rotated, the K and V projections write the
-        layer's cache (K rotated) directly, then only the attention runs."""
+        projection leaves Q rotated, one K/V projection writes the layer's
+        cache (K rotated) directly, then only the attention runs."""
         w = self.w
         ly, wt = self.layers[index], self.weights[index]
         b = ly.buf
         star.star_rmsnorm(x, wt["gamma"], self.h, self.eps)
         star.star_linear_rope(self.h, wt["wq"], self.q, w.D, True, w.L, 0, w.theta, 0,
                               self.gemm_ws)
-        star.star_linear_rope(self.h, wt["wk"], b.k_cache, w.D, True, w.L, 0, w.theta, w.Lcap,
-                              self.gemm_ws)
-        star.star_linear_rope(self.h, wt["wv"], b.v_cache, w.D, False, w.L, 0, w.theta, w.Lcap,
-                              self.gemm_ws)
+        star.star_linear_kv_cache(self.h, self.w_kv[index], b.k_cache, b.v_cache, w.L, 0,
+                                  w.theta, self.gemm_ws)
         star.star_phase1_encode_rotated(self.q, b.o, b.k_cache, b.v_cache, w.L, w.block_len,
                                         w.anchor_len, b.ws1)
         star.star_linear(b.o, wt["wo"], x, accumulate=True, workspace=self.gemm_ws)

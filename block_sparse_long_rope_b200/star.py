@@ -297,6 +297,26 @@ def star_linear_rope(x, w, y, head_dim, rotate, seq_len, pos0, theta, cache_rows
     return y
 
 
+def star_linear_kv_cache(x, w_kv, k_cache, v_cache, seq_len, pos0, theta, workspace,
+                         stream=None):
+    """A layer's K and V projections in one GEMM (w_kv = [Wk; Wv], [2N, K]):
+    rotated keys into k_cache, values into v_cache (head-major [B, Hkv,
+    cache_rows, D]), token t of each sequence in cache row t."""
+    for t, n in ((x, "x"), (w_kv, "w_kv"), (k_cache, "k_cache"), (v_cache, "v_cache")):
+        _bf16(t, n)
+        if not t.is_contiguous():
+            raise ValueError(f"{n} must be contiguous")
+    N2, K = w_kv.shape
+    M = x.numel() // K
+    D, rows = k_cache.shape[3], k_cache.shape[2]
+    lib = _abi.load()
+    _abi.check(lib.star_linear_kv_cache(_ptr(x), _ptr(w_kv), _ptr(k_cache), _ptr(v_cache), M,
+                                        N2 // 2, K, D, int(seq_len), int(pos0), float(theta),
+                                        rows, _ptr(workspace),
+                                        workspace.numel() * workspace.element_size(),
+                                        _stream(stream)))
+
+
 def star_linear_rope_workspace_bytes(seq_len, head_dim, rotate) -> int:
     return int(_abi.load().star_linear_rope_workspace_bytes(int(seq_len), int(head_dim),
                                                             1 if rotate else 0))

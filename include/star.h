@@ -397,6 +397,24 @@ star_status star_linear(const void* x, const void* w, void* y, int M, int N, int
  * star_linear.
  */
 size_t star_linear_rope_workspace_bytes(int seq_len, int head_dim, int rotate);
+
+/*
+ * star_linear_kv_cache — a layer's K and V projections as one GEMM, written
+ * straight into its KV cache: w_kv[2N, K] holds the K projection's N rows
+ * and then the V projection's N rows (N = Hkv * head_dim). With
+ * p = bf16(x[M, K] * w_kv^T): columns [0, N) are the keys, rotated as
+ * star_linear_rope rotates them (position pos0 + t), into k_cache; columns
+ * [N, 2N) are the values, unrotated, into v_cache; both caches head-major
+ * [M / seq_len, Hkv, cache_rows, head_dim], token t of sequence b in row t.
+ * The bits equal star_linear_rope(K, rotate = 1) and star_linear_rope(V,
+ * rotate = 0) on the two halves; one launch fills the GPU better than two
+ * narrow ones. cache_rows >= seq_len; workspace as star_linear_rope with
+ * rotate = 1. Errors as star_linear_rope.
+ */
+star_status star_linear_kv_cache(const void* x, const void* w_kv, void* k_cache, void* v_cache,
+                                 int M, int N, int K, int head_dim, int seq_len, int64_t pos0,
+                                 double theta, int cache_rows, void* workspace,
+                                 size_t workspace_bytes, void* cuda_stream);
 star_status star_linear_rope(const void* x, const void* w, void* y, int M, int N, int K,
                              int head_dim, int rotate, int seq_len, int64_t pos0, double theta,
                              int cache_rows, void* workspace, size_t workspace_bytes,

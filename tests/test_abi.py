@@ -293,6 +293,16 @@ def test_stack_calls_validation(lib):
     assert lib.star_linear_rope_workspace_bytes(4096, 128, 1) == 256 + 4096 * 64 * 8
     assert lib.star_linear_rope_workspace_bytes(5, 64, 1) == 256 + 5 * 32 * 8
     assert lib.star_linear_rope_workspace_bytes(4096, 128, 0) == 256
+    # K/V projection into the caches: whole heads, cache rows >= seq_len, both caches given
+    def kv(N=128, hd=64, S=4, rows=8, vc=FAKE, ws=FAKE, wsb=1 << 20):
+        return lib.star_linear_kv_cache(FAKE, FAKE, FAKE, vc, 8, N, 64, hd, S, 0, 1e4, rows, ws,
+                                        wsb, NULL)
+    assert kv(hd=96) == UNSUPPORTED
+    assert kv(N=96) == INVALID
+    assert kv(rows=3) == INVALID
+    assert kv(vc=NULL) == INVALID
+    assert kv(vc=ODD) == INVALID
+    assert kv(wsb=256) == INVALID         # no room for the cos/sin table
 
 
 def test_phase1_rotated_validation(lib):

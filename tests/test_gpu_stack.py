@@ -112,6 +112,18 @@ def test_linear_rope_equals_linear_then_rope(B, S, H, D, K, pos0):
     # and against the oracle's correctly rounded rotation of the bf16 projection
     rot = orc.rope(p.cpu(), np.arange(pos0, pos0 + S), theta, round_out=True)
     np.testing.assert_array_equal(to64(q), rot)
+    # K and V in one GEMM (w_kv = [Wk; Wv]): the same bits as the two calls
+    wv = inputs.randn_bf16((N, K), 13, scale=K ** -0.5).to(dev)
+    pv = torch.empty((B, S, H, D), dtype=torch.bfloat16, device=dev)
+    star.star_linear(x, wv, pv, workspace=ws)
+    kc2 = torch.full_like(kc, float("nan"))
+    vc2 = torch.full_like(vc, float("nan"))
+    star.star_linear_kv_cache(x, torch.cat([w, wv]).contiguous(), kc2, vc2, S, pos0, theta, ws)
+    star.star_device_status(ws)
+    torch.cuda.synchronize()
+    assert torch.equal(kc2[:, :, :S], ref.permute(0, 2, 1, 3))
+    assert torch.equal(vc2[:, :, :S], pv.permute(0, 2, 1, 3))
+    assert torch.isnan(kc2[:, :, S:].float()).all() and torch.isnan(vc2[:, :, S:].float()).all()
 
 
 def test_stack_encode_and_steps_match_the_oracle():
