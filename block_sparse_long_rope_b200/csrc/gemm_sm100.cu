@@ -18,13 +18,17 @@
 //                (row m = b * seq_len + t lands in cache row t of sequence b),
 //                rotated (K) or not (V)
 //
-// Design: a persistent kernel, one CTA per SM, 192 threads.
+// Design: a persistent kernel, one CTA per SM, 320 threads.
 //   warp 0     TMA producer: A (128 x 64) and B (256 x 64) tiles, 128-byte
 //              swizzle, through a 4-stage shared-memory ring
 //   warp 1     TMEM allocator and single-thread tcgen05.mma issuer
 //              (M = 128, N = 256, K = 16 per instruction, both operands
 //              K-major)
-//   warps 2-5  epilogue: thread = output row = TMEM lane
+//   warps 2-9  epilogue, two warpgroups: thread = output row = TMEM lane,
+//              warps 2-5 take the tile's columns 0-127 and warps 6-9 the
+//              columns 128-255 (the RoPE epilogue would otherwise outlast a
+//              tile's main loop: one warpgroup left the tensor pipe idle 37%
+//              of the time)
 // The fp32 accumulator is double-buffered in tensor memory (2 x 256
 // columns), so a tile's epilogue overlaps the next tile's MMAs. Tiles are
 // taken in row-major order (m outer, n inner), so the CTAs in flight share
@@ -39,7 +43,8 @@ namespace star {
 
 namespace {
 
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;
+constexpr int kEpiThreads = 256;  // warps 2-9
 constexpr int kBM = 128, kBN = 256, kBK = 64, kGemmStages = 4;
 constexpr int kATile = kBM * kBK * 2;  // 16 KB
 constexpr int kBTile = kBN * kBK * 2;  // 32 KB
@@ -107,15 +112,29 @@ __device__ __forceinline__ void store_plain32(const GemmParams& p, const OutRow&
   }
 }
 
-// 32 bf16 values (bits in the low 16 of each word) to four 16-byte vectors at column n.
-__device__ __forceinline__ void store_bits32(const GemmParams& p, const OutRow& o, int n,
-                                             const uint32_t (&h)[32]) {
+// 16 bf16 values (bits in the low 16 of each word) to two 16-byte vectors at column n.
+__device__ __forceinline__ void store_bits16(const GemmParams& p, const OutRow& o, int n,
+                                             const uint32_t (&h)[16]) {
 #pragma unroll
-  for (int v = 0; v < 4; ++v) {
+  for (int v = 0; v < 2; ++v) {
     __nv_bfloat16* dst = out_at(p, o, n + 8 * v);
     uint32_t w[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) w[j] = h[8 * v + 2 * j] | (h[8 * v + 2 * j + 1] << 16);
+    *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// 16 accumulator columns -> bf16, two 16-byte vectors at column n (no residual).
+__device__ __forceinline__ void store_plain16(const GemmParams& p, const OutRow& o, int n,
+                                              const uint32_t (&r)[16]) {
+#pragma unroll
+  for (int v = 0; v < 2; ++v) {
+    __nv_bfloat16* dst = out_at(p, o, n + 8 * v);
+    uint32_t w[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      w[j] = pack_bf16x2(__uint_as_float(r[8 * v + 2 * j]), __uint_as_float(r[8 * v + 2 * j + 1]));
     *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
@@ -146,7 +165,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&acc_full[x], 1);
-      mbar_init(&acc_empty[x], 128);
+      mbar_init(&acc_empty[x], kEpiThreads);
     }
     mbar_init(done, 1);
     fence_barrier_init();
@@ -223,8 +242,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31 (warps 2-5 -> 2,3,0,1)
+    const int quad = warp & 3;  // TMEM lanes 32*quad .. 32*quad+31 (warps 2-9 -> 2,3,0,1,2,3,0,1)
     const int row = 32 * quad + lane;
+    const int half = (warp - 2) >> 2;  // which 128 of the tile's 256 columns
+    constexpr int kHalfN = kBN / 2;
     int lt = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++lt) {
       const int ab = lt & 1, use = lt >> 1;
@@ -238,7 +259,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
       const uint32_t tb = tmem + (static_cast<uint32_t>(32 * quad) << 16) + ab * kAccCols;
       if constexpr (RD == 0) {
 #pragma unroll 1
-        for (int c = 0; c < kBN / 32; ++c) {
+        for (int c = half * (kHalfN / 32); c < (half + 1) * (kHalfN / 32); ++c) {
           uint32_t r[32];
           tmem_ld32(tb + 32 * c, r);
           tmem_wait_ld();
@@ -246,17 +267,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
           if (mvalid && n0 + 32 * c < p.N) store_plain32(p, orow, n0 + 32 * c, r);
         }
       } else {
-        // heads of RD columns; pair (i, i + RD/2); 32 frequencies at a time,
+        // heads of RD columns; pair (i, i + RD/2); 16 frequencies at a time,
         // their fp32 cos/sin read once from the call's table (built by
-        // rope_table_kernel) and shared by the tile's heads
+        // rope_table_kernel) and shared by this warpgroup's heads
         const int t = mvalid ? m % p.seq_len : 0;
         const long long pos = p.pos0 + t;
 #pragma unroll 1
-        for (int fc = 0; fc < RD / 64; ++fc) {
-          float c32[32], s32[32];
-          const float4* tab = reinterpret_cast<const float4*>(p.rope_tab + static_cast<size_t>(t) * (RD / 2) + 32 * fc);
+        for (int fc = 0; fc < RD / 32; ++fc) {
+          float c32[16], s32[16];
+          const float4* tab = reinterpret_cast<const float4*>(p.rope_tab + static_cast<size_t>(t) * (RD / 2) + 16 * fc);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
+          for (int j = 0; j < 8; ++j) {
             const float4 cs = tab[j];
             c32[2 * j] = cs.x;
             s32[2 * j] = cs.y;
@@ -264,35 +285,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1) gemm_kernel(const __grid_cons
             s32[2 * j + 1] = cs.w;
           }
 #pragma unroll 1
-          for (int h = 0; h < kBN / RD; ++h) {
-            const int col = h * RD + 32 * fc;  // first-half column of this chunk
+          for (int h = half * (kHalfN / RD); h < (half + 1) * (kHalfN / RD); ++h) {
+            const int col = h * RD + 16 * fc;  // first-half column of this chunk
             if (n0 + h * RD >= p.N) break;     // warp-uniform
-            uint32_t x[32], y[32];
-            tmem_ld32(tb + col, x);
-            tmem_ld32(tb + col + RD / 2, y);
+            uint32_t x[16], y[16];
+            tmem_ld16(tb + col, x);
+            tmem_ld16(tb + col + RD / 2, y);
             tmem_wait_ld();
-            reg_fence32(x);
-            reg_fence32(y);
+            reg_fence16(x);
+            reg_fence16(y);
             if (n0 + h * RD >= p.n_split) {  // a V head of a K/V projection: no rotation
               if (mvalid) {
-                store_plain32(p, orow2, n0 + col - p.n_split, x);
-                store_plain32(p, orow2, n0 + col + RD / 2 - p.n_split, y);
+                store_plain16(p, orow2, n0 + col - p.n_split, x);
+                store_plain16(p, orow2, n0 + col + RD / 2 - p.n_split, y);
               }
               continue;
             }
             if (mvalid) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j) {
+              for (int j = 0; j < 16; ++j) {
                 // the stored (bf16) projection is what gets rotated
                 const float a = bf16_round(__uint_as_float(x[j]));
                 const float b = bf16_round(__uint_as_float(y[j]));
                 const uint32_t pr = rope_rotate_pair_bf16_at(a, b, c32[j], s32[j], pos,
-                                                             p.inv_freq[32 * fc + j]);
+                                                             p.inv_freq[16 * fc + j]);
                 x[j] = pr & 0xFFFFu;
                 y[j] = pr >> 16;
               }
-              store_bits32(p, orow, n0 + col, x);
-              store_bits32(p, orow, n0 + col + RD / 2, y);
+              store_bits16(p, orow, n0 + col, x);
+              store_bits16(p, orow, n0 + col + RD / 2, y);
             }
           }
         }

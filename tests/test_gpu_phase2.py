@@ -198,3 +198,41 @@ def test_overlapping_decode_graph_at_16k_matches_eager_and_oracle():
                              new[2].cpu(), t, w.theta, np.zeros(w.Hq), hh, np.zeros(w.Hq))
     assert max_abs(to64(o_g)[0, 0], go) <= TOL_O
     assert max_abs(to64(lse_g)[0, :, 0], gl) <= TOL_LSE
+
+
+def test_decode_reads_q_written_just_before_it():
+    """Decode calls reuse one q/k/v buffer that a kernel rewrites right before
+    each call (as a projection would). The decode kernel may start while the
+    kernel before it drains (programmatic dependent launch), so it must read
+    q only after that kernel has ended: every step must see its own new
+    token, checked against the oracle's global attention."""
+    from block_sparse_long_rope_b200 import inputs
+    from block_sparse_long_rope_b200.configs import Workload
+    from block_sparse_long_rope_b200.pipeline import StarLayer
+
+    w = Workload(index=71, name="decode-q-rewrite", B=1, Hq=32, Hkv=8, D=128, theta=5.0e5,
+                 L=8192, block_len=2048, anchor_len=2048, Tq=0, Tdec=6)
+    ctx = inputs.make_context(w.B, w.L, w.Hq, w.Hkv, w.D, w.index, device="cuda")
+    new = inputs.make_new_tokens(w.B, w.Tdec, w.Hq, w.Hkv, w.D, w.index, device="cuda")
+    layer = StarLayer(w)
+    layer.encode(*ctx)
+    qb = torch.empty((w.B, 1, w.Hq, w.D), dtype=torch.bfloat16, device="cuda")
+    kb = torch.empty((w.B, 1, w.Hkv, w.D), dtype=torch.bfloat16, device="cuda")
+    vb = torch.empty_like(kb)
+    outs = []
+    for s in range(w.Tdec):
+        # the writes of this step's token land just before the decode launch
+        qb.copy_(new[0][:, s:s + 1])
+        kb.copy_(new[1][:, s:s + 1])
+        vb.copy_(new[2][:, s:s + 1])
+        o, lse = layer.attend(qb, kb, vb, s)
+        outs.append((o.clone(), lse.clone()))
+    torch.cuda.synchronize()
+    star.star_device_status(layer.buf.ws2)
+    hh = np.arange(w.Hq)
+    for s, (o, lse) in enumerate(outs):
+        go, gl = orc.global_rows(new[0][:, s:s + 1].cpu(), ctx[1].cpu(), ctx[2].cpu(),
+                                 new[1].cpu(), new[2].cpu(), s, w.theta, np.zeros(w.Hq), hh,
+                                 np.zeros(w.Hq))
+        assert max_abs(to64(o)[0, 0], go) <= TOL_O, f"step {s}"
+        assert max_abs(to64(lse)[0, :, 0], gl) <= TOL_LSE, f"step {s}"
