@@ -168,3 +168,31 @@ def test_phase1_against_unrounded_oracle(name):
     assert d_rnd[0] <= TOL_O and d_rnd[1] <= TOL_LSE
     assert d_f64[0] <= TOL_O
     assert excess <= TOL_LSE
+
+
+@pytest.mark.parametrize("shape", [(1, 1000, 4, 2, 64, 300, 100, 1e4), (2, 1536, 8, 2, 128, 512, 512, 5e5)],
+                         ids=["L1000b300a100D64", "B2L1536b512D128"])
+def test_phase1_rotated_entry_equals_encode(shape):
+    """star_phase1_encode_rotated on a Q rotated by star_rope and a cache
+    whose rows [0, L) hold the rotated keys and the values gives the bits of
+    star_phase1_encode on the pre-RoPE inputs (the same attention kernel)."""
+    B, L, Hq, Hkv, D, b, a, theta = shape
+    q = rand_bf16((B, L, Hq, D), seed=L + 31)
+    k = rand_bf16((B, L, Hkv, D), seed=L + 32)
+    v = rand_bf16((B, L, Hkv, D), seed=L + 33)
+    o_ref, lse_ref, kc_ref, vc_ref = encode(q, k, v, b, a, theta, Lcap=L + 3)
+    qr = torch.empty_like(q)
+    star.star_rope(q, qr, theta)
+    kc = torch.full_like(kc_ref, float("nan"))
+    vc = torch.full_like(vc_ref, float("nan"))
+    star.star_rope(k, kc[:, :, :L].permute(0, 2, 1, 3), theta)
+    vc[:, :, :L] = v.permute(0, 2, 1, 3)
+    o = torch.empty_like(q)
+    lse = torch.empty_like(lse_ref)
+    ws = star.alloc_workspace(256)
+    star.star_phase1_encode_rotated(qr, o, kc, vc, L, b, a, ws, lse=lse)
+    star.star_device_status(ws)
+    torch.cuda.synchronize()
+    assert torch.equal(kc[:, :, :L], kc_ref[:, :, :L])
+    assert torch.equal(o, o_ref)
+    assert torch.equal(lse, lse_ref)

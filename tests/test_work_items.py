@@ -72,6 +72,7 @@ PHASE1 = [  # (B, Hq, Hkv, L, b, a)
     (1, 4, 2, 500, 64, 64),
     (1, 2, 1, 100, 1, 1),
     (1, 16, 2, 1300, 650, 650),
+    (2, 16, 4, 1100, 256, 256),   # items ordered KV-head-major over two sequences
 ]
 
 
