@@ -80,13 +80,17 @@ struct AttnGeom {
   __host__ __device__ int qtiles_last() const { return ceil_div(L - (n - 1) * b, kTileM); }
 
   // ---- Phase 1 -------------------------------------------------------------
-  // Items are ordered longest first: by descending query-tile index j (work
-  // grows with j), and within one j blocks 1..n-1 before block 0 (block 0
-  // has no anchor tiles).
-  __host__ __device__ int phase1_items() const {
+  // Items are ordered by (batch, KV head) first, so the CTAs in flight read
+  // the same anchor and own-block K/V tiles and L2 serves them (at 1M tokens
+  // a head's anchor is 64 MB, all eight heads' K/V 4 GB). Within one KV head
+  // they run longest first: by descending query-tile index j (work grows
+  // with j), within one j blocks 1..n-1 before block 0 (block 0 has no
+  // anchor tiles), then the head pairs of the GQA group.
+  __host__ __device__ int phase1_pairs() const {  // (block, query tile) pairs
     int nf = qtiles_full(), nl = qtiles_last();
-    return ((nf - nl) * (n - 1) + nl * n) * groups();
+    return (nf - nl) * (n - 1) + nl * n;
   }
+  __host__ __device__ int phase1_items() const { return phase1_pairs() * groups(); }
   __host__ __device__ void group_decode(int gi, WorkItem* w) const {
     int g = Hq / Hkv, per_kv = g / hpc;
     w->b = gi / (Hkv * per_kv);
@@ -95,24 +99,28 @@ struct AttnGeom {
     w->slot0 = w->kvh * g + (rem % per_kv) * hpc;
   }
   __host__ __device__ WorkItem phase1_item(int item) const {
-    int G = groups();
+    const int per_kv = (Hq / Hkv) / hpc;  // head pairs (groups) of one KV head
+    const int chunk = phase1_pairs() * per_kv;
+    const int bk = item / chunk;          // b * Hkv + kvh
+    const int in = item % chunk;
     int nf = qtiles_full(), nl = qtiles_last();
-    int top = (nf - nl) * (n - 1) * G;
-    int j, i, gi;
-    if (item < top) {
-      int per = (n - 1) * G;
-      int jj = item / per, rem = item % per;
+    int top = (nf - nl) * (n - 1) * per_kv;
+    int j, i, sg;
+    if (in < top) {
+      int per = (n - 1) * per_kv;
+      int jj = in / per, rem = in % per;
       j = nf - 1 - jj;
-      i = (rem / G + 1) % (n - 1);
-      gi = rem % G;
+      i = (rem / per_kv + 1) % (n - 1);
+      sg = rem % per_kv;
     } else {
-      int it = item - top;
-      int per = n * G;
+      int it = in - top;
+      int per = n * per_kv;
       int jj = it / per, rem = it % per;
       j = nl - 1 - jj;
-      i = (rem / G + 1) % n;
-      gi = rem % G;
+      i = (rem / per_kv + 1) % n;
+      sg = rem % per_kv;
     }
+    const int gi = bk * per_kv + sg;
     WorkItem w;
     group_decode(gi, &w);
     int s = i * b, e = imin(s + b, L);
