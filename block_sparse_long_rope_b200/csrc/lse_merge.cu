@@ -142,18 +142,21 @@ __global__ void debug_wait_probe_kernel(int* status, unsigned long long limit_ns
 // blocks): lane s takes block s's sub-split LSEs, its max m_s and sum
 // z_s = sum_k e^(l_k - m_s), hence its LSE m_s + log z_s; the tail split's
 // LSE is read as written; M is the max over the splits. Pass 2 (lanes over
-// D) reads every sub-split output once, four blocks' rows issued before they
-// are used: a block's partial is sum_k e^(l_k - lse_s) o_k (written to
-// part_o), and the merged row adds every split with weight e^(lse_s - M)
+// D) reads every sub-split output once, the rows of several blocks issued
+// before they are used (kSub = the sub-split count rounded up to 1, 2 or 4;
+// a lane holds 4 rows at D = 128 and 8 at D = 64, 64 registers, so four
+// CTAs fit on an SM and 4096 rows run in one wave): a block's partial is
+// sum_k e^(l_k - lse_s) o_k (written to part_o), and the merged row adds
+// every split with weight e^(lse_s - M)
 // [pith 2WVXFXZ2, minor comment on Algorithm 2]. Fixed order, deterministic.
-template <int D>
-__global__ void __launch_bounds__(256) chunk_finish_kernel(
+template <int D, int kSub>
+__global__ void __launch_bounds__(256, 4) chunk_finish_kernel(
     const float* __restrict__ sub_o, const float* __restrict__ sub_lse, int nsub, int n, int tail,
     float* __restrict__ part_o, float* __restrict__ part_lse, __nv_bfloat16* __restrict__ o,
     float* __restrict__ lse, int B, int T, int Hq) {
   constexpr int kPer = D / 32;
-  constexpr int kMaxSub = 4;   // sub-splits per block (the cut rule makes at most 4)
-  constexpr int kBlk = 4;      // blocks whose rows are loaded together
+  constexpr int kMaxSub = kSub;  // nsub <= kSub <= 4 (the cut rule makes at most 4)
+  constexpr int kBlk = (D == 128 ? 4 : 8) / kSub;  // blocks whose rows are loaded together
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) / 32;
   const int lane = threadIdx.x % 32;
   if (warp >= B * Hq * T) return;
@@ -271,12 +274,20 @@ cudaError_t launch_chunk_finish(const float* sub_o, const float* sub_lse, int ns
   if (rows == 0) return cudaSuccess;
   const int threads = 256;
   const unsigned blocks = static_cast<unsigned>((rows * 32 + threads - 1) / threads);
-  if (D == 128)
-    chunk_finish_kernel<128><<<blocks, threads, 0, stream>>>(sub_o, sub_lse, nsub, n, tail, part_o,
-                                                             part_lse, o, lse, B, T, Hq);
-  else
-    chunk_finish_kernel<64><<<blocks, threads, 0, stream>>>(sub_o, sub_lse, nsub, n, tail, part_o,
-                                                            part_lse, o, lse, B, T, Hq);
+#define STAR_CHUNK_FINISH(DD, KS)                                                              \
+  chunk_finish_kernel<DD, KS><<<blocks, threads, 0, stream>>>(sub_o, sub_lse, nsub, n, tail,    \
+                                                              part_o, part_lse, o, lse, B, T, Hq)
+  const int ks = nsub <= 1 ? 1 : (nsub == 2 ? 2 : 4);
+  if (D == 128) {
+    if (ks == 1) STAR_CHUNK_FINISH(128, 1);
+    else if (ks == 2) STAR_CHUNK_FINISH(128, 2);
+    else STAR_CHUNK_FINISH(128, 4);
+  } else {
+    if (ks == 1) STAR_CHUNK_FINISH(64, 1);
+    else if (ks == 2) STAR_CHUNK_FINISH(64, 2);
+    else STAR_CHUNK_FINISH(64, 4);
+  }
+#undef STAR_CHUNK_FINISH
   return cudaGetLastError();
 }
 
