@@ -316,9 +316,9 @@ def cold_decode(layer, call, reps, dev, world):
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(reps)]
     for a, b in evs:
-        # a spin of ~100 us puts the host ahead of the device, so the events
+        # a spin of ~0.5 ms puts the host ahead of the device, so the events
         # time the call's kernels and not the host's Python between them
-        torch.cuda._sleep(200_000)
+        torch.cuda._sleep(1_000_000)
         flush_l2(flush)
         a.record(stream)
         layer.attend(q2, k2, v2, tail)
