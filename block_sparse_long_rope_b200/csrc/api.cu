@@ -104,12 +104,13 @@ EncodeTiledFn encode_fn() {
 }
 
 // rank-4 map over a token-major [B, rows, H, D] bf16 buffer; box {64, 1, 128, 1}
-star_status map_token_major(CUtensorMap* m, const void* base, int B, int rows, int H, int D) {
+star_status map_token_major(CUtensorMap* m, const void* base, int B, int rows, int H, int D,
+                            int box_rows = 128) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return fail(STAR_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)B};
   cuuint64_t strides[3] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2, (cuuint64_t)rows * H * D * 2};
-  cuuint32_t box[4] = {64, 1, 128, 1};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t es[4] = {1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
                    box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -419,6 +420,7 @@ star_status phase1_run(const void* q, const void* k, const void* v, void* o, voi
   ap.geom.Hq = Hq;
   ap.geom.Hkv = Hkv;
   ap.geom.hpc = (g % 2 == 0) ? 2 : 1;
+  ap.geom.hps = 1;
   ap.geom.L = L;
   ap.geom.b = block_len;
   ap.geom.a = ext ? 0 : anchor_len;
@@ -636,13 +638,16 @@ star_status phase2_run(const void* q, const void* k, const void* v, int T, void*
 
   star::AttnParams ap;
   memset(&ap, 0, sizeof ap);
-  if ((s = map_token_major(&ap.tmQ, qrot, B, T, Hq, D)) != STAR_OK) return s;
+  // chunks of at most 64 tokens put two heads in each 128-row tile
+  const int hps = star::chunk_heads_per_slot(T, Hq, Hkv);
+  if ((s = map_token_major(&ap.tmQ, qrot, B, T, Hq, D, 128 / hps)) != STAR_OK) return s;
   if ((s = map_cache(&ap.tmK, k_cache, B * Hkv, Lcap, valid, D, 128)) != STAR_OK) return s;
   if ((s = map_cache(&ap.tmV, v_cache, B * Hkv, Lcap, valid, D, 128)) != STAR_OK) return s;
   ap.geom.B = B;
   ap.geom.Hq = Hq;
   ap.geom.Hkv = Hkv;
   ap.geom.hpc = (g % 2 == 0) ? 2 : 1;
+  ap.geom.hps = hps;
   ap.geom.L = L;
   ap.geom.b = block_len;
   ap.geom.a = 0;

@@ -111,6 +111,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const WorkItem w = (kMode == 0) ? p.geom.phase1_item(blockIdx.x) : p.geom.phase2_item(blockIdx.x);
   const int hpc = p.geom.hpc;
+  // heads per 128-row tile: 2 for query chunks of at most 64 tokens (rows
+  // 0-63 head slot0 + 2x, rows 64-127 the next head), else 1
+  const int hps = (kMode == 1) ? p.geom.hps : 1;
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -174,10 +177,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
       }
       mbar_arrive_expect_tx(q_full, hpc * C::kTile);
       for (int x = 0; x < hpc; ++x)
+        for (int hh = 0; hh < hps; ++hh)  // a 64-row box per head when hps = 2
 #pragma unroll
-        for (int hd = 0; hd < D / 64; ++hd)
-          tma_load_4d(sm + C::kOffQ + x * C::kTile + hd * C::kHalf, &p.tmQ, q_full, hd * 64,
-                      w.slot0 + x, w.q_lo, w.b);
+          for (int hd = 0; hd < D / 64; ++hd)
+            tma_load_4d(sm + C::kOffQ + x * C::kTile + hd * C::kHalf + hh * (C::kHalf / 2), &p.tmQ,
+                        q_full, hd * 64, w.slot0 + x * hps + hh, w.q_lo, w.b);
       const int bz = w.b * p.geom.Hkv + w.kvh;
       int issued_k = 0, issued_v = 0;
       int csi = 0, cti = 0;  // span cursor
@@ -279,7 +283,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     const uint32_t lane_bits = static_cast<uint32_t>(qw * 32) << 16;
     const uint32_t tS = tmem + lane_bits + C::col_s(x);
     const uint32_t tO = tmem + lane_bits + C::col_o(x);
-    const int qrow = w.q_lo + row;
+    const int hrow = (hps == 2) ? (row >> 6) : 0;  // which head of the tile
+    const int qrow = w.q_lo + ((hps == 2) ? (row & 63) : row);
     const int qpos = w.pos_base + qrow;
     const int min_pos = w.pos_base + w.q_lo;
     const float c = p.scale_log2;
@@ -388,7 +393,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
     // ---------------------------------------------------------------- epilogue
     if (ok && mbar_wait(o_full, 0, &abort_flag, p.status)) {
       tc_fence_after();
-      const int head = w.slot0 + x;
+      const int head = w.slot0 + x * hps + hrow;
       const bool valid = qrow < w.q_hi;
       const float inv = (l_run > 0.f) ? 1.f / l_run : 0.f;
       const int b = w.b;

@@ -64,10 +64,19 @@ struct WorkItem {
   }
 };
 
+// Query chunks of at most 64 tokens fill a 128-row tile with two heads of
+// the same GQA group (rows 0-63 one head, 64-127 the next), so no MMA row
+// is left empty; needs four heads per KV head (two tiles of two heads).
+__host__ __device__ __forceinline__ int chunk_heads_per_slot(int T, int Hq, int Hkv) {
+  return (T <= 64 && (Hq / Hkv) % 4 == 0) ? 2 : 1;
+}
+
 // Geometry shared by the two attention modes. Query heads are handled
-// `hpc` at a time (the heads of one GQA group that share every K/V tile).
+// `hpc` tiles at a time (the heads of one GQA group that share every K/V
+// tile), each tile holding `hps` heads (2 only for short query chunks).
 struct AttnGeom {
-  int B, Hq, Hkv, hpc;  // hpc: query heads per CTA (1 or 2)
+  int B, Hq, Hkv, hpc;  // hpc: query tiles (head slots) per CTA (1 or 2)
+  int hps;              // heads per tile: 1, or 2 (64 rows each; Phase 2 only)
   int L, b, a;          // context length, block length, anchor length
   int n;                // context blocks = ceil(L / b)
   // Phase 2 only
@@ -75,7 +84,8 @@ struct AttnGeom {
   int tail;             // 1: the call's cache holds the tail split (new tokens)
   int nsub, sub_len;    // query chunks: sub-splits per context block, keys each
 
-  __host__ __device__ int groups() const { return B * Hkv * ((Hq / Hkv) / hpc); }
+  __host__ __device__ int heads_per_item() const { return hpc * hps; }
+  __host__ __device__ int groups() const { return B * Hkv * ((Hq / Hkv) / heads_per_item()); }
   __host__ __device__ int qtiles_full() const { return ceil_div(imin(b, L), kTileM); }
   __host__ __device__ int qtiles_last() const { return ceil_div(L - (n - 1) * b, kTileM); }
 
@@ -92,14 +102,14 @@ struct AttnGeom {
   }
   __host__ __device__ int phase1_items() const { return phase1_pairs() * groups(); }
   __host__ __device__ void group_decode(int gi, WorkItem* w) const {
-    int g = Hq / Hkv, per_kv = g / hpc;
+    int g = Hq / Hkv, per_kv = g / heads_per_item();
     w->b = gi / (Hkv * per_kv);
     int rem = gi % (Hkv * per_kv);
     w->kvh = rem / per_kv;
-    w->slot0 = w->kvh * g + (rem % per_kv) * hpc;
+    w->slot0 = w->kvh * g + (rem % per_kv) * heads_per_item();
   }
   __host__ __device__ WorkItem phase1_item(int item) const {
-    const int per_kv = (Hq / Hkv) / hpc;  // head pairs (groups) of one KV head
+    const int per_kv = (Hq / Hkv) / heads_per_item();  // head groups of one KV head
     const int chunk = phase1_pairs() * per_kv;
     const int bk = item / chunk;          // b * Hkv + kvh
     const int in = item % chunk;

@@ -81,7 +81,8 @@ inline int chunk_subsplits(int B, int Hq, int Hkv, int T, int L, int block_len, 
   if (!with_tail || L % block_len != 0) return 1;
   const int n = L / block_len;
   const int g = Hq / Hkv, hpc = (g % 2 == 0) ? 2 : 1;
-  const long long per_split = (long long)B * Hkv * (g / hpc) * ceil_div(T, 128);
+  const int hpi = hpc * chunk_heads_per_slot(T, Hq, Hkv);
+  const long long per_split = (long long)B * Hkv * (g / hpi) * ceil_div(T, 128);
   if ((n + 1) * per_split >= kWave) return 1;
   int nsub = (int)std::min<long long>(4, (kWave - per_split) / (n * per_split));
   while (nsub > 1 && block_len % (nsub * 128) != 0) --nsub;

@@ -1,8 +1,10 @@
 // Host build of the attention kernels' work decomposition (star_index.cuh),
 // for CPU tests: the same header the kernels include, with the CUDA function
 // qualifiers defined away. Each call builds the geometry the way the
-// library's entry points do (hpc = 2 query heads per item when the GQA group
-// size is even, else 1) and writes one work item as 8 + 2 * 6 integers:
+// library's entry points do (hpc = 2 query-head tiles per item when the GQA
+// group size is even, else 1; two heads per tile for query chunks of at most
+// 64 tokens when the group has 4 or more heads) and writes one work item as
+// 8 + 2 * 6 integers:
 // b, kvh, slot0, q_lo, q_hi, pos_base, split, nspan, then per span key0,
 // ntiles, lo, hi, causal, src.
 #define __host__
@@ -19,6 +21,7 @@ static AttnGeom geom(int B, int Hq, int Hkv, int L, int b, int a) {
   g.Hq = Hq;
   g.Hkv = Hkv;
   g.hpc = ((Hq / Hkv) % 2 == 0) ? 2 : 1;
+  g.hps = 1;
   g.L = L;
   g.b = b;
   g.a = a;
@@ -40,6 +43,11 @@ extern "C" {
 
 int wi_hpc(int Hq, int Hkv) { return ((Hq / Hkv) % 2 == 0) ? 2 : 1; }
 
+// query heads per Phase-2 item (two tiles of two heads for chunks of <= 64 tokens)
+int wi_phase2_heads_per_item(int Hq, int Hkv, int T) {
+  return wi_hpc(Hq, Hkv) * star::chunk_heads_per_slot(T, Hq, Hkv);
+}
+
 int wi_phase1_items(int B, int Hq, int Hkv, int L, int b, int a) {
   return geom(B, Hq, Hkv, L, b, a).phase1_items();
 }
@@ -51,6 +59,7 @@ void wi_phase1_item(int B, int Hq, int Hkv, int L, int b, int a, int item, int* 
 static AttnGeom geom2(int B, int Hq, int Hkv, int L, int b, int T, int tail_len, int with_tail,
                       int nsub) {
   AttnGeom g = geom(B, Hq, Hkv, L, b, 0);
+  g.hps = star::chunk_heads_per_slot(T, Hq, Hkv);
   g.T = T;
   g.tail_len = tail_len;
   g.tail = with_tail;

@@ -116,13 +116,16 @@ PHASE2 = [  # (B, Hq, Hkv, L, b, T, tail_len, with_tail, nsub)
     (1, 32, 8, 4096, 1024, 128, 0, 1, 2),
     (1, 32, 8, 16384, 4096, 128, 0, 1, 4),
     (1, 4, 2, 1024, 256, 40, 3, 0, 1),   # a shard without the tail split
+    (2, 32, 8, 2048, 512, 64, 9, 1, 2),  # 64 tokens: two heads per tile, sub-splits
+    (1, 8, 1, 1100, 256, 33, 0, 1, 1),   # ragged last block, two heads per tile
 ]
 
 
 @pytest.mark.parametrize("geo", PHASE2, ids=[f"L{g[3]}b{g[4]}T{g[5]}sub{g[8]}tail{g[7]}" for g in PHASE2])
 def test_phase2_items_cover_each_split_row_once_with_exactly_its_keys(lib, geo):
     B, Hq, Hkv, L, b, T, tail_len, with_tail, nsub = geo
-    hpc = lib.wi_hpc(Hq, Hkv)
+    hpi = lib.wi_phase2_heads_per_item(Hq, Hkv, T)  # 4 for <= 64 tokens and groups of 4+
+    assert hpi == lib.wi_hpc(Hq, Hkv) * (2 if T <= 64 and (Hq // Hkv) % 4 == 0 else 1)
     n = -(-L // b)
     sub_len = b // nsub
     n_items = lib.wi_phase2_items(*geo)
@@ -136,7 +139,8 @@ def test_phase2_items_cover_each_split_row_once_with_exactly_its_keys(lib, geo):
         assert 0 <= s < nsplit and it["pos_base"] == L + tail_len
         assert it["q_lo"] < it["q_hi"] <= T and it["q_hi"] - it["q_lo"] <= TILE
         rows = np.arange(it["q_lo"], it["q_hi"])
-        for h in range(it["slot0"], it["slot0"] + hpc):
+        assert it["slot0"] % hpi == 0 and it["kvh"] == it["slot0"] // (Hq // Hkv)
+        for h in range(it["slot0"], it["slot0"] + hpi):
             count[it["b"], h, s, rows] += 1
         keys = np.arange(nkeys)
         if s < n * nsub:
