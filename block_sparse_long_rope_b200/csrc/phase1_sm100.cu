@@ -314,14 +314,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1) attn_kernel(const __grid_cons
       const bool full_vis =
           key0 >= lo && key0 + 128 <= hi && (!causal || key0 + 127 <= min_pos);
       if (!full_vis) {
+        // the row's visible keys in this tile are one run [vlo, vhi) of
+        // tile columns: one unsigned compare per column
+        const int vlo = imax(lo - key0, 0);
+        const int vhi = imin(imin(hi - key0, 128), causal ? qpos - key0 + 1 : 128);
+        const uint32_t span = static_cast<uint32_t>(imax(vhi - vlo, 0));
 #pragma unroll
         for (int q = 0; q < 4; ++q)
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const int key = key0 + 32 * q + j;
-            const bool vis = key >= lo && key < hi && (!causal || key <= qpos);
-            if (!vis) sr[q][j] = __float_as_uint(-INFINITY);
-          }
+          for (int j = 0; j < 32; ++j)
+            if (static_cast<uint32_t>(32 * q + j - vlo) >= span) sr[q][j] = __float_as_uint(-INFINITY);
       }
       // row max: eight independent chains of 3-input max, then a tree (one
       // chain of 128 dependent max operations would dominate the latency)
