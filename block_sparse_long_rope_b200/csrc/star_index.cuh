@@ -90,12 +90,12 @@ struct AttnGeom {
   __host__ __device__ int qtiles_last() const { return ceil_div(L - (n - 1) * b, kTileM); }
 
   // ---- Phase 1 -------------------------------------------------------------
-  // Items are ordered by (batch, KV head) first, so the CTAs in flight read
-  // the same anchor and own-block K/V tiles and L2 serves them (at 1M tokens
-  // a head's anchor is 64 MB, all eight heads' K/V 4 GB). Within one KV head
-  // they run longest first: by descending query-tile index j (work grows
-  // with j), within one j blocks 1..n-1 before block 0 (block 0 has no
-  // anchor tiles), then the head pairs of the GQA group.
+  // Items are ordered by (batch, KV head) first, then block by block: the
+  // anchor-carrying blocks 1..n-2, the last block, then block 0 (no anchor,
+  // the shortest items). The CTAs in flight then read one KV head's anchor
+  // and one block, 2 x 64 MB at 1M tokens, which L2 mostly keeps. Inside a
+  // block the query tiles run longest first (descending index j, work grows
+  // with j), the head groups of a tile next to each other.
   __host__ __device__ int phase1_pairs() const {  // (block, query tile) pairs
     int nf = qtiles_full(), nl = qtiles_last();
     return (nf - nl) * (n - 1) + nl * n;
@@ -113,23 +113,29 @@ struct AttnGeom {
     const int chunk = phase1_pairs() * per_kv;
     const int bk = item / chunk;          // b * Hkv + kvh
     const int in = item % chunk;
-    int nf = qtiles_full(), nl = qtiles_last();
-    int top = (nf - nl) * (n - 1) * per_kv;
-    int j, i, sg;
-    if (in < top) {
-      int per = (n - 1) * per_kv;
-      int jj = in / per, rem = in % per;
-      j = nf - 1 - jj;
-      i = (rem / per_kv + 1) % (n - 1);
-      sg = rem % per_kv;
+    const int nf = qtiles_full(), nl = qtiles_last();
+    int i, j, r;
+    if (n == 1) {
+      i = 0;
+      r = in;
+      j = nl - 1 - r / per_kv;
     } else {
-      int it = in - top;
-      int per = n * per_kv;
-      int jj = it / per, rem = it % per;
-      j = nl - 1 - jj;
-      i = (rem / per_kv + 1) % n;
-      sg = rem % per_kv;
+      const int full = (n - 2) * nf * per_kv, last = nl * per_kv;
+      if (in < full) {  // blocks 1..n-2
+        i = 1 + in / (nf * per_kv);
+        r = in % (nf * per_kv);
+        j = nf - 1 - r / per_kv;
+      } else if (in < full + last) {  // block n-1
+        i = n - 1;
+        r = in - full;
+        j = nl - 1 - r / per_kv;
+      } else {  // block 0
+        i = 0;
+        r = in - full - last;
+        j = nf - 1 - r / per_kv;
+      }
     }
+    const int sg = r % per_kv;
     const int gi = bk * per_kv + sg;
     WorkItem w;
     group_decode(gi, &w);
