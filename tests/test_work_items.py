@@ -108,6 +108,38 @@ def test_phase1_items_cover_each_row_once_with_exactly_its_visible_keys(lib, geo
     assert (count == 1).all()
 
 
+@pytest.mark.parametrize("geo", [(2, 16, 4, 1100, 256, 256), (1, 32, 8, 1 << 20, 131072, 131072),
+                                 (1, 8, 2, 1536, 512, 128)],
+                         ids=["B2-ragged", "llama8b-1m", "a<b"])
+def test_phase1_item_order_keeps_one_kv_head_and_block_together(lib, geo):
+    """The L2-friendly order: items run (batch, KV head) by (batch, KV head);
+    inside one, block by block (1..n-2, the last block, then block 0); inside
+    a block, query tiles longest first."""
+    B, Hq, Hkv, L, b, a = geo
+    n = -(-L // b)
+    n_items = lib.wi_phase1_items(B, Hq, Hkv, L, b, a)
+    want_blocks = list(range(1, n - 1)) + ([n - 1] if n > 1 else []) + [0]
+    step = max(1, n_items // 20000)  # the 1M shape has 131072 items: a sample and its neighbours
+    idx = range(0, n_items) if n_items <= 20000 else sorted(
+        set(range(0, n_items, step)) | set(range(1, n_items, step)))
+    order = []
+    for i in idx:
+        it = _item(lib.wi_phase1_item, B, Hq, Hkv, L, b, a, i)
+        order.append((i, it["b"] * Hkv + it["kvh"], it["q_lo"] // b, it["q_lo"]))
+    # (batch, KV head) never decreases
+    assert all(x[1] <= y[1] for x, y in zip(order, order[1:]))
+    for bk in sorted({o[1] for o in order}):
+        seq = [o for o in order if o[1] == bk]
+        blk_seq = [o[2] for o in seq]
+        # blocks appear as contiguous runs, in the stated order
+        runs = [blk_seq[0]] + [y for x, y in zip(blk_seq, blk_seq[1:]) if y != x]
+        assert runs == [blk for blk in want_blocks if blk in set(blk_seq)], runs[:12]
+        # inside a block, query tiles never move forward
+        for x, y in zip(seq, seq[1:]):
+            if x[2] == y[2] and y[0] == x[0] + 1:
+                assert y[3] <= x[3]
+
+
 PHASE2 = [  # (B, Hq, Hkv, L, b, T, tail_len, with_tail, nsub)
     (1, 4, 1, 2048, 512, 16, 0, 1, 1),
     (2, 4, 2, 1000, 300, 20, 5, 1, 1),
