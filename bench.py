@@ -984,7 +984,7 @@ def run_sharded(args, w, rank, world, local_rank):
     return line
 
 
-def run_reference(args, w, rank):
+def run_reference(args, w, rank, world=1):
     """Reference arm: the fp64 oracle as it stands, on the host cores. A full
     step of a long-context workload would take hours to days on a CPU, so
     each of the K steps times a bounded random sample of that step's work
@@ -994,6 +994,10 @@ def run_reference(args, w, rank):
     minutes."""
     if rank != 0:
         return None
+    # the oracle runs on all the host's cores: a torchrun launch sets
+    # OMP_NUM_THREADS=1 for every rank, and the other ranks do no work here
+    # (read by the oracle's OpenMP runtime when the oracle library loads)
+    os.environ["OMP_NUM_THREADS"] = str(os.cpu_count() or 1)
     per_step = max(1.0, min(args.ref_budget, 150.0 / max(1, args.steps + args.warmup)))
     host = _host_inputs(w, 0)
     for _ in range(args.warmup):
@@ -1010,13 +1014,14 @@ def run_reference(args, w, rank):
     est_step = sum(est) / len(est)
     value = w.B * w.L / est_step
     return {
-        "metric": METRIC, "value": round(value, 3), "unit": "tok/s", "n_gpus": 1,
+        "metric": METRIC, "value": round(value, 3), "unit": "tok/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(est_step * 1e3, 1),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic N(0,1) bf16 Q/K/V (seeded)", "impl": "reference",
         "extrapolated": True,
         "ran": (f"{args.steps} timed samples of about {per_step:.1f} s each ({spent:.1f} s of "
-                f"oracle work, {wall:.1f} s wall); ms_per_step is the step time extrapolated "
+                f"oracle work, {wall:.1f} s wall) on rank 0's host cores (the launch's "
+                f"{world} rank(s); no GPU work); ms_per_step is the step time extrapolated "
                 "from the samples, not a timed step"),
         "seconds_timed": round(spent, 2),
         "config": {"workload": w.name, "B": w.B, "L": w.L, "Hq": w.Hq, "Hkv": w.Hkv, "D": w.D,
@@ -1084,7 +1089,7 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         # rank 0 alone times the oracle on the host cores; other ranks exit 0
-        line = run_reference(args, w, rank)
+        line = run_reference(args, w, rank, world)
         if line is not None:
             print(json.dumps(line), flush=True)
         return
