@@ -122,6 +122,9 @@ FLOWS = [
     (1, 700, 16, 2, 128, 256, 256, 5e5, [2, 3, 1, 1]),                # g=8: R=16 decode, R=24 chunk
     (1, 900, 2, 2, 128, 200, 200, 5e5, [1, 130, 1]),                  # g=1: T=130 = 2 query tiles
     (1, 4096, 32, 8, 128, 1024, 1024, 5e5, [128, 1, 1]),              # 8B layer shape, short context
+    (1, 4096, 32, 8, 128, 1024, 1024, 5e5, [64, 1, 1]),               # 64-token chunk: two heads per tile, sub-splits
+    (2, 2048, 16, 4, 128, 512, 512, 5e5, [33, 1]),                    # two sequences, ragged packed chunk
+    (1, 2048, 64, 8, 128, 512, 512, 5e5, [40, 1]),                    # 70B head layout (g = 8), packed chunk
 ]
 
 
