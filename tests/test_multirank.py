@@ -103,3 +103,23 @@ def test_multi_gpu_runs_default_to_the_sharded_deployment():
     assert bench.resolve_mode(None, 8) == "sharded"
     assert bench.resolve_mode("replicas", 8) == "replicas"
     assert bench.resolve_mode("sharded", 1) == "sharded"
+
+
+def test_code_digest_ignores_comments_and_layout(tmp_path, monkeypatch):
+    a = tmp_path / "a.cu"
+    b = tmp_path / "b.cu"
+    a.write_text("int f(int x) {\n  return x + 1;  // one more\n}\n/* block\ncomment */\n")
+    b.write_text("int f(int x){return x+1;}\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.code_digest(["a.cu"]) == bench.code_digest(["b.cu"])
+    b.write_text("int f(int x){return x+2;}\n")
+    assert bench.code_digest(["a.cu"]) != bench.code_digest(["b.cu"])
+
+
+def test_committed_phase1_traffic_records_match_the_kernel_sources():
+    """The bench line's roofline `traffic` comes from an ncu capture recorded
+    under profiles/; it is reported only while the kernel sources are the
+    ones captured (comments aside)."""
+    for wl in ("llama8b-1m", "llama8b-16k"):
+        t = bench.phase1_traffic(wl)
+        assert isinstance(t, int) and t > 0, wl
